@@ -1,0 +1,452 @@
+#!/usr/bin/env python
+"""Decode-step benchmark of the RTPurbo attention hot path on B200.
+
+One step = one decode step of the workload: every layer's rtp_decode_step (indexer scoring,
+sort-free top-p, compaction, sparse + window attention) for every sequence of the batch.
+Prints ONE JSON line (rank 0).
+
+  python bench.py [--gpus N --steps K --warmup W] [--workload ctx_1m] [--top-p 0.9]
+  python bench.py --impl reference ...   # the fp64 CPU oracle on the host cores
+
+Timing: the step is captured once as a CUDA graph (all layers), replayed W times untimed,
+then K times between CUDA events on the launch stream, bracketed by a barrier and a
+device synchronisation; the max over ranks is reported. The step reads several GB from HBM,
+far more than the 126 MB L2, so no flush is needed between steps.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import subprocess
+import sys
+import tempfile
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "decode steps/s and effective HBM GB/s (% of roofline) at 128K–1M ctx"
+ROW_BYTES = 2 * 128 * 2      # one token's K and V rows (bf16, head_dim 128)
+IDX_BYTES = 16 * 2           # one token's indexer key (fp16, 16 dims)
+
+
+def _peaks():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            p = json.load(f)
+        return float(p["hbm_gbs"]), "measured"
+    except Exception:
+        return 6650.0, "fallback"
+
+
+class ClockSampler:
+    """nvidia-smi clock / throttle sampling during the timed region."""
+    QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        try:
+            fd, self.path = tempfile.mkstemp(suffix=".csv")
+            os.close(fd)
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.QUERY}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+
+    def stop(self) -> dict:
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        rows = []
+        with open(self.path) as f:
+            for line in f:
+                parts = [x.strip() for x in line.split(",")]
+                if len(parts) >= 9:
+                    rows.append(parts)
+        os.unlink(self.path)
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
+        sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
+        smax = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i in range(4) if r[5 + i] == "Active"})
+        return {"sm_mhz": float(np.median(sm)) if sm else None,
+                "sm_max_mhz": max(smax) if smax else None, "reasons": reasons,
+                "samples": len(rows)}
+
+
+def step_bytes(plan, sel_counts) -> tuple[int, int, int]:
+    """Algorithmic HBM bytes of one step: indexer keys of every retrieval head (N x 32 B),
+    selected K/V rows (|S| x 512 B) and window K/V rows (|T| x 512 B).
+    Returns (total, attend_bytes, indexer_bytes)."""
+    idx = att = 0
+    for l in range(plan.num_layers):
+        for b in range(plan.batch):
+            N = int(plan.seq_lens[b])
+            for h in range(plan.num_kv_heads):
+                att += int(sel_counts[l][b, h]) * ROW_BYTES
+                if plan.retrieval[l, h]:
+                    idx += N * IDX_BYTES
+    return idx + att, att, idx
+
+
+def cpu_sample_layers(plan):
+    """A bounded sample of the workload for the CPU oracle: one layer with a broad (diffuse or
+    flat) retrieval query, one with a concentrated one and one with local heads only."""
+    from head_wise_sparse_retrieval_b200 import workloads as W
+    pick = []
+    for cond in (lambda l: ((plan.kind[l] == W.KIND_DIFFUSE) | (plan.kind[l] == W.KIND_FLAT)).any(),
+                 lambda l: (plan.kind[l] == W.KIND_CONC).any(),
+                 lambda l: not plan.retrieval[l].any()):
+        for l in range(plan.num_layers):
+            if cond(l) and l not in pick:
+                pick.append(l)
+                break
+    return pick or [0]
+
+
+def oracle_layer_seconds(plan, li, layer, top_p, threads):
+    """Time the oracle (fp64 C, OpenMP over heads) on one layer; host copies excluded."""
+    import oracle
+    from head_wise_sparse_retrieval_b200 import workloads as W
+    args = dict(q=W.to_host_u16(li.q), q_idx=W.to_host_u16(li.q_idx),
+                k_cache=W.to_host_u16(li.k_cache), v_cache=W.to_host_u16(li.v_cache),
+                k_idx=W.to_host_u16(li.k_idx), seq_lens=li.seq_lens.cpu().numpy(),
+                retrieval_mask=plan.retrieval[layer])
+    t = time.perf_counter()
+    _, nsel = oracle.decode_layer(**args, top_p=float(np.float32(top_p)), window=plan.window,
+                                  sinks=plan.sinks, num_threads=threads)
+    return time.perf_counter() - t, nsel
+
+
+def oracle_step_bytes(plan, layer_fn):
+    """Algorithmic bytes of a full step from the oracle's own token sets: it scores every
+    retrieval head and runs the histogram top-p on it; local heads use the window set."""
+    import oracle
+    from head_wise_sparse_retrieval_b200 import workloads as W
+    p = float(np.float32(plan.top_p))
+    total = 0
+    for l in range(plan.num_layers):
+        li = layer_fn(l) if plan.retrieval[l].any() else None
+        for b in range(plan.batch):
+            N = int(plan.seq_lens[b])
+            for h in range(plan.num_kv_heads):
+                if plan.retrieval[l, h]:
+                    s = oracle.indexer_scores(W.to_host_u16(li.q_idx[b, h]),
+                                              W.to_host_u16(li.k_idx[b, h, :N]), 0.25)
+                    total += N * IDX_BYTES + oracle.hist_topp(s, p).sel.size * ROW_BYTES
+                else:
+                    total += oracle.window_sink_set(N, plan.window, plan.sinks).size * ROW_BYTES
+        del li
+    return total
+
+
+def oracle_sample(plan, layer_fn, layers, threads):
+    """Oracle seconds and algorithmic bytes on the sampled layers."""
+    secs, nbytes = [], []
+    for l in layers:
+        li = layer_fn(l)
+        dt, nsel = oracle_layer_seconds(plan, li, l, plan.top_p, threads)
+        secs.append(dt)
+        nbytes.append(sum(int(nsel[b, k]) * ROW_BYTES +
+                          (int(plan.seq_lens[b]) * IDX_BYTES if plan.retrieval[l, k] else 0)
+                          for b in range(plan.batch) for k in range(plan.num_kv_heads)))
+        del li
+    return secs, nbytes
+
+
+def run_reference(args, plan, rank, world):
+    """--impl reference: the fp64 CPU oracle on the host cores, each step a bounded sample of
+    the same workload (one sampled layer), its time scaled to a full step by bytes."""
+    if rank != 0:
+        return
+    import torch
+    import oracle
+    from head_wise_sparse_retrieval_b200 import workloads as W
+    dev = "cuda" if torch.cuda.is_available() else "cpu"
+    layers = cpu_sample_layers(plan)
+    threads = oracle.max_threads()
+    cores = min(threads, plan.batch * plan.num_kv_heads)
+    layer_fn = lambda l: W.make_layer(plan, l, dev)
+    full = oracle_step_bytes(plan, layer_fn)
+    cache = {l: layer_fn(l) for l in layers}
+    times = []
+    for i in range(args.warmup + args.steps):
+        l = layers[i % len(layers)]
+        secs, nbytes = oracle_sample(plan, lambda _l: cache[_l], [l], threads)
+        if i >= args.warmup:
+            times.append(secs[0] * full / max(nbytes[0], 1))
+    sec_per_step = float(np.mean(times))
+    value = 1.0 / sec_per_step
+    sample = (f"one layer per step, cycling layers {layers} of {plan.name} (broad-query, "
+              f"concentrated-query, local-only); fp64 oracle time scaled to a full step by "
+              f"algorithmic bytes ({full} B per step from the oracle's own selections)")
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "steps/s",
+            "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": sec_per_step * 1e3, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": plan.name, "layers": plan.num_layers, "batch": plan.batch,
+                       "ctx": plan.ctx, "top_p": plan.top_p},
+            "cpu_baseline": {"value": value, "unit": "steps/s", "cores": cores,
+                             "kind": "oracle", "sample": sample},
+            "e2e": {"value": value, "unit": "steps/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["rtp", "reference"], default="rtp")
+    ap.add_argument("--workload", default="ctx_1m",
+                    choices=["tiny", "one_layer", "batch_decode", "long_context", "ctx_1m"])
+    ap.add_argument("--top-p", type=float, default=None)
+    ap.add_argument("--layers", type=int, default=None, help="fewer layers (debug only)")
+    ap.add_argument("--ctx", type=int, default=None, help="other context length (debug only)")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-dense", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    args = ap.parse_args()
+    args.warmup = max(args.warmup, 3)
+
+    import torch
+    import torch.distributed as dist
+    from head_wise_sparse_retrieval_b200 import rtp
+    from head_wise_sparse_retrieval_b200 import workloads as W
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        torch.cuda.set_device(local)
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=600),
+                                device_id=torch.device("cuda", local))
+
+    plan = W.plan(args.workload, top_p=args.top_p, num_layers=args.layers, ctx=args.ctx)
+
+    if args.impl == "reference":
+        run_reference(args, plan, rank, world)
+        if world > 1:
+            dist.barrier()
+            dist.destroy_process_group()
+        return
+
+    rtp.load()
+    dev = torch.device("cuda", local if world > 1 else 0)
+    torch.cuda.set_device(dev)
+    L, B, Hq, Hkv = plan.num_layers, plan.batch, plan.num_q_heads, plan.num_kv_heads
+
+    t_gen = time.perf_counter()
+    layers = [W.make_layer(plan, l, dev) for l in range(L)]
+    torch.cuda.synchronize()
+    t_gen = time.perf_counter() - t_gen
+    outs = [torch.empty((B, Hq, 128), dtype=torch.float32, device=dev) for _ in range(L)]
+    cnts = [torch.empty((B, Hkv), dtype=torch.int32, device=dev) for _ in range(L)]
+    h = rtp.Handle(rtp.config_for(plan), dev.index)
+    views = [rtp.layer_from(li) for li in layers]
+    stream = torch.cuda.Stream(device=dev)
+
+    def step(dense=False):
+        for l in range(L):
+            if dense:
+                h.dense_decode(views[l], outs[l], stream=stream)
+            else:
+                h.decode_step(l, views[l], plan.retrieval[l], plan.top_p, outs[l], cnts[l],
+                              stream=stream)
+
+    # eager step: checks the path end to end and gives the token-set sizes
+    with torch.cuda.stream(stream):
+        step()
+    torch.cuda.synchronize()
+    status = h.device_status()
+    if status:
+        raise SystemExit(f"device status 0x{status:x} after the eager step")
+    sel = [c.cpu().numpy() for c in cnts]
+    total_bytes, attend_bytes, idx_bytes = step_bytes(plan, sel)
+    launches_per_step = sum(4 if plan.retrieval[l].any() else 1 for l in range(L))
+
+    # capture the whole step as one CUDA graph
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=stream):
+        step()
+    for _ in range(args.warmup):
+        g.replay()
+    torch.cuda.synchronize()
+
+    sampler = ClockSampler(dev.index if world == 1 else local)
+    if rank == 0:
+        sampler.start()
+        time.sleep(0.3)
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    e0.record(stream)
+    for _ in range(args.steps):
+        g.replay()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    clocks = sampler.stop() if rank == 0 else {}
+    ms = e0.elapsed_time(e1) / args.steps
+    if world > 1:
+        t = torch.tensor([ms], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms = float(t.item())
+    del g
+
+    # per-kernel durations (CUDA events around each launch on the launch stream)
+    h.profile(True)
+    prof_steps = max(3, min(args.steps, 10))
+    acc = {k: [0.0, 0] for k in rtp.KERNEL_CLASSES}
+    for _ in range(prof_steps):
+        with torch.cuda.stream(stream):
+            step()
+        for k, (t_ms, n) in h.profile_read().items():
+            acc[k][0] += t_ms
+            acc[k][1] += n
+    h.profile(False)
+    kern = {k: {"ms_total_per_step": v[0] / prof_steps, "launches_per_step": v[1] / prof_steps}
+            for k, v in acc.items()}
+    att_ms = acc["attend"][0] / max(acc["attend"][1], 1)
+    att_bytes_per_launch = attend_bytes / L
+    hbm, peak_kind = _peaks()
+    att_gbs = att_bytes_per_launch / (att_ms * 1e-3) / 1e9
+
+    # dense decode on the same caches (the speedup denominator)
+    dense = None
+    if not args.no_dense:
+        gd = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(gd, stream=stream):
+            step(dense=True)
+        for _ in range(3):
+            gd.replay()
+        torch.cuda.synchronize()
+        nd = max(3, min(args.steps, 5))
+        d0 = torch.cuda.Event(enable_timing=True)
+        d1 = torch.cuda.Event(enable_timing=True)
+        d0.record(stream)
+        for _ in range(nd):
+            gd.replay()
+        d1.record(stream)
+        torch.cuda.synchronize()
+        dms = d0.elapsed_time(d1) / nd
+        dense_bytes = sum(int(plan.seq_lens[b]) * ROW_BYTES for b in range(B)) * Hkv * L
+        dense = {"ms_per_step": dms, "speedup": dms / ms,
+                 "effective_gbs": dense_bytes / (dms * 1e-3) / 1e9}
+        del gd
+
+    # end to end through the host-buffer entry point: pinned host queries in, outputs out
+    e2e = None
+    if not args.no_e2e:
+        q_h = torch.stack([li.q for li in layers]).cpu().pin_memory()
+        qi_h = torch.stack([li.q_idx for li in layers]).cpu().pin_memory()
+        seq_h = layers[0].seq_lens.cpu().pin_memory()
+        out_h = torch.empty((L, B, Hq, 128), dtype=torch.float32).pin_memory()
+        masks = plan.retrieval.astype(np.uint8)
+        for _ in range(2):
+            h.decode_step_host(q_h, qi_h, seq_h, views, masks, plan.top_p, out_h, stream=stream)
+        ne = max(3, min(args.steps, 10))
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize()
+        x0 = torch.cuda.Event(enable_timing=True)
+        x1 = torch.cuda.Event(enable_timing=True)
+        x0.record(stream)
+        for _ in range(ne):
+            h.decode_step_host(q_h, qi_h, seq_h, views, masks, plan.top_p, out_h, stream=stream)
+        x1.record(stream)
+        torch.cuda.synchronize()
+        xms = x0.elapsed_time(x1) / ne
+        if world > 1:
+            t = torch.tensor([xms], device=dev)
+            dist.all_reduce(t, op=dist.ReduceOp.MAX)
+            xms = float(t.item())
+        e2e = {"value": world * 1e3 / xms, "unit": "steps/s",
+               "h2d_bytes_per_step": int(q_h.numel() * 2 + qi_h.numel() * 2 + seq_h.numel() * 4),
+               "d2h_bytes_per_step": int(out_h.numel() * 4), "ms_per_step": xms}
+
+    # CPU baseline: the oracle on a bounded sample of the workload (rank 0, N = 1 only)
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        import oracle
+        picks = cpu_sample_layers(plan)
+        threads = oracle.max_threads()
+        full = oracle_step_bytes(plan, lambda l: layers[l])
+        secs_l, bytes_l = oracle_sample(plan, lambda l: layers[l], picks, threads)
+        secs, sbytes = sum(secs_l), sum(bytes_l)
+        est = secs * full / max(sbytes, 1)
+        cpu = {"value": 1.0 / est, "unit": "steps/s",
+               "cores": int(min(threads, B * Hkv)), "kind": "oracle",
+               "sample": (f"layers {picks} of {plan.name} (broad-query, concentrated-query and "
+                          f"local-only layers), {secs:.1f} s of fp64 oracle time, scaled to a "
+                          f"full step by algorithmic bytes"),
+               "host_threads": threads}
+
+    value = world * 1e3 / ms
+    eff_gbs = total_bytes / (ms * 1e-3) / 1e9
+    n_sel = [int(s[b, k]) for l, s in enumerate(sel) for b in range(B) for k in range(Hkv)
+             if plan.retrieval[l, k]]
+    line = {
+        "metric": METRIC, "value": value, "unit": "steps/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic",
+        "config": {"workload": plan.name, "layers": L, "batch": B, "ctx": plan.ctx,
+                   "q_heads": Hq, "kv_heads": Hkv, "head_dim": 128, "idx_dim": 16,
+                   "retrieval_kv_heads": int(plan.retrieval.sum()), "top_p": plan.top_p,
+                   "window": plan.window, "sinks": plan.sinks,
+                   "l2": "no flush: each step reads several GB (> 126 MB L2)",
+                   "parallelism": "replicas" if world > 1 else "single GPU",
+                   "timing": "CUDA graph of all layers, CUDA events on the launch stream"},
+        "effective_gbs": eff_gbs,
+        "roofline_frac_step": eff_gbs / hbm,
+        "algorithmic_bytes_per_step": total_bytes,
+        "bytes_breakdown": {"indexer": idx_bytes, "attend_kv": attend_bytes},
+        "roofline": {"bound": "hbm", "kernel": "attend_kernel", "achieved": att_gbs,
+                     "peak": hbm, "peak_kind": peak_kind, "unit": "GB/s",
+                     "frac": att_gbs / hbm, "traffic": None,
+                     "per_launch_ms": att_ms, "algorithmic_bytes_per_launch": att_bytes_per_launch},
+        "kernels": kern,
+        "selection": {"retrieval_heads": len(n_sel),
+                      "mean_selected": float(np.mean(n_sel)) if n_sel else 0.0,
+                      "max_selected": int(max(n_sel)) if n_sel else 0},
+        "dense": dense,
+        "e2e": e2e,
+        "cpu_baseline": cpu,
+        "gpu_launches": launches_per_step * args.steps,
+        "clocks": clocks,
+        "setup_s": t_gen,
+    }
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    h.close()
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,585 @@
+// rtp_api.cu -- host side of librtp: argument checks, workspace, launches (C-ABI of rtp.h).
+#include <cmath>
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <vector>
+
+#include "rtp.h"
+#include "rtp_device.cuh"
+#include "rtp_kernels.h"
+
+using namespace rtp;
+
+struct rtp_handle {
+  rtp_config cfg;
+  int device = 0;
+  int num_sms = 0;
+  int G = 0;
+  int attend_grid = 0;
+  size_t attend_smem = 0;
+  void* ws_mem = nullptr;
+  size_t ws_bytes = 0;
+  Workspace ws{};
+  // staging for rtp_decode_step_host
+  void* stage_q = nullptr;
+  void* stage_qidx = nullptr;
+  int* stage_seq = nullptr;
+  float* stage_out = nullptr;
+  // bookkeeping of the last rtp_decode_step, for the debug getters
+  bool last_valid = false;
+  cudaStream_t last_stream = nullptr;
+  int last_nret = 0;
+  short last_slot_of_kvh[kMaxKvHeads];
+  // kernel profiling (rtp_profile_enable)
+  bool prof = false;
+  std::vector<cudaEvent_t> prof_ev;   // 2 per launch
+  std::vector<int> prof_kind;
+  int prof_used = 0;
+  bool prof_overflow = false;
+};
+
+namespace {
+
+thread_local char g_err[256] = "";
+
+rtp_status fail(rtp_status s, const char* fmt, ...) {
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(g_err, sizeof g_err, fmt, ap);
+  va_end(ap);
+  return s;
+}
+
+rtp_status ok() {
+  g_err[0] = '\0';
+  return RTP_OK;
+}
+
+rtp_status cuda_fail(cudaError_t e, const char* what) {
+  return fail(RTP_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+rtp_status check_config(const rtp_config* c) {
+  if (!c) return fail(RTP_ERR_INVALID_ARG, "config is NULL");
+  if (c->num_layers < 1) return fail(RTP_ERR_INVALID_ARG, "num_layers must be >= 1");
+  if (c->batch < 1) return fail(RTP_ERR_INVALID_ARG, "batch must be >= 1");
+  if (c->num_kv_heads < 1 || c->num_kv_heads > kMaxKvHeads)
+    return fail(RTP_ERR_INVALID_ARG, "num_kv_heads must be in [1, %d]", kMaxKvHeads);
+  if (c->num_q_heads < 1 || c->num_q_heads % c->num_kv_heads != 0)
+    return fail(RTP_ERR_INVALID_ARG, "num_q_heads must be a positive multiple of num_kv_heads");
+  if ((long long)c->batch * c->num_kv_heads > kMaxAttendHeads)
+    return fail(RTP_ERR_UNSUPPORTED, "batch * num_kv_heads must be <= %d", kMaxAttendHeads);
+  const int G = c->num_q_heads / c->num_kv_heads;
+  if (G > kMaxGroup) return fail(RTP_ERR_UNSUPPORTED, "GQA group size %d > %d", G, kMaxGroup);
+  if (c->head_dim != kHeadDim) return fail(RTP_ERR_UNSUPPORTED, "head_dim must be 128");
+  if (c->idx_dim != kIdxDim) return fail(RTP_ERR_UNSUPPORTED, "idx_dim must be 16");
+  if (c->num_bins != kBins) return fail(RTP_ERR_UNSUPPORTED, "num_bins must be 256");
+  if (c->max_ctx < 1 || c->max_ctx > (1 << 28))
+    return fail(RTP_ERR_INVALID_ARG, "max_ctx must be in [1, 2^28]");
+  if (c->window < 1) return fail(RTP_ERR_INVALID_ARG, "window must be >= 1");
+  if (c->sinks < 0) return fail(RTP_ERR_INVALID_ARG, "sinks must be >= 0");
+  if (c->window > (1 << 28) || c->sinks > (1 << 28))
+    return fail(RTP_ERR_INVALID_ARG, "window and sinks must be <= 2^28");
+  if (!(c->idx_range > 0.f) || !std::isfinite(c->idx_range))
+    return fail(RTP_ERR_INVALID_ARG, "idx_range must be finite and > 0");
+  if (!(c->idx_scale > 0.f) || !std::isfinite(c->idx_scale))
+    return fail(RTP_ERR_INVALID_ARG, "idx_scale must be finite and > 0");
+  if (!(c->attn_scale > 0.f) || !std::isfinite(c->attn_scale))
+    return fail(RTP_ERR_INVALID_ARG, "attn_scale must be finite and > 0");
+  return RTP_OK;
+}
+
+struct WsPlan {
+  size_t off[20];
+  size_t total;
+};
+
+// Byte offsets of the workspace arrays (each 256-byte aligned).
+WsPlan plan_workspace(const rtp_config* c, int attend_grid) {
+  const size_t slots = (size_t)c->batch * c->num_kv_heads;
+  const size_t nmax = (size_t)c->max_ctx;
+  const size_t nsc = (nmax + kScoreChunk - 1) / kScoreChunk;
+  const size_t nsel = (nmax + kSelChunk - 1) / kSelChunk;
+  const size_t sizes[] = {
+      slots * nmax * 4,                      // 0 scores
+      slots * nsc * 4,                       // 1 chunk_max
+      slots * kBins * 8,                     // 2 hist
+      slots * 4,                             // 3 s_max
+      slots * 4,                             // 4 bstar
+      slots * 8,                             // 5 mass_total
+      slots * nmax * 4,                      // 6 sel_idx
+      slots * nsel * 4,                      // 7 chunk_cnt
+      slots * (nsel + 1) * 4,                // 8 chunk_off
+      slots * 4,                             // 9 sel_total
+      slots * 4,                             // 10 sel_n
+      slots * 4,                             // 11 ticket_hist
+      slots * 4,                             // 12 ticket_compact
+      slots * 4,                             // 13 ticket_attend
+      ((size_t)attend_grid + slots) * kMaxGroup * kPartStride * 4,  // 14 partials
+      256,                                   // 15 status
+  };
+  WsPlan p{};
+  size_t at = 0;
+  for (size_t i = 0; i < sizeof sizes / sizeof sizes[0]; ++i) {
+    p.off[i] = at;
+    at = round_up(at + sizes[i], 256);
+  }
+  p.total = at;
+  return p;
+}
+
+template <typename Kernel>
+cudaError_t launch_pdl(Kernel k, dim3 grid, dim3 block, size_t smem, cudaStream_t s,
+                       const LayerArgs& a, const Workspace& w) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, k, a, w);
+}
+
+rtp_status check_io(const rtp_handle* h, const rtp_layer_io* io, bool need_idx) {
+  if (!io) return fail(RTP_ERR_INVALID_ARG, "io is NULL");
+  if (!io->q || !io->k_cache || !io->v_cache || !io->seq_lens || !io->out)
+    return fail(RTP_ERR_INVALID_ARG, "q, k_cache, v_cache, seq_lens and out must be non-NULL");
+  if (!aligned16(io->q) || !aligned16(io->k_cache) || !aligned16(io->v_cache) ||
+      !aligned16(io->out))
+    return fail(RTP_ERR_INVALID_ARG, "q, k_cache, v_cache and out must be 16-byte aligned");
+  if (((uintptr_t)io->seq_lens & 3u) || ((uintptr_t)io->sel_count & 3u))
+    return fail(RTP_ERR_INVALID_ARG, "seq_lens and sel_count must be 4-byte aligned");
+  if (need_idx) {
+    if (!io->q_idx || !io->k_idx)
+      return fail(RTP_ERR_INVALID_ARG, "q_idx and k_idx are required for retrieval heads");
+    if (!aligned16(io->q_idx) || !aligned16(io->k_idx))
+      return fail(RTP_ERR_INVALID_ARG, "q_idx and k_idx must be 16-byte aligned");
+    if (!(io->top_p > 0.f && io->top_p <= 1.f))
+      return fail(RTP_ERR_INVALID_ARG, "top_p must be in (0, 1]");
+  }
+  (void)h;
+  return RTP_OK;
+}
+
+LayerArgs make_args(const rtp_handle* h, const rtp_layer_io* io) {
+  LayerArgs a;
+  memset(&a, 0, sizeof a);
+  a.q = static_cast<const __nv_bfloat16*>(io->q);
+  a.q_idx = static_cast<const __half*>(io->q_idx);
+  a.k_cache = static_cast<const __nv_bfloat16*>(io->k_cache);
+  a.v_cache = static_cast<const __nv_bfloat16*>(io->v_cache);
+  a.k_idx = static_cast<const __half*>(io->k_idx);
+  a.seq_lens = io->seq_lens;
+  a.out = io->out;
+  a.sel_count = io->sel_count;
+  a.B = h->cfg.batch;
+  a.Hq = h->cfg.num_q_heads;
+  a.Hkv = h->cfg.num_kv_heads;
+  a.G = h->G;
+  a.max_ctx = h->cfg.max_ctx;
+  a.window = h->cfg.window;
+  a.sinks = h->cfg.sinks;
+  a.top_p = io->top_p;
+  a.idx_scale = h->cfg.idx_scale;
+  a.attn_scale_log2 = (float)((double)h->cfg.attn_scale * 1.4426950408889634);
+  a.bin_scale = (float)((double)kBins / (double)h->cfg.idx_range);
+  for (int k = 0; k < kMaxKvHeads; ++k) a.slot_of_kvh[k] = -1;
+  return a;
+}
+
+constexpr int kProfCapacity = 1024;
+
+// Launches one kernel, bracketed by profiling events when the handle has profiling enabled.
+template <typename Kernel>
+cudaError_t launch_one(rtp_handle* h, int kind, Kernel k, dim3 grid, dim3 block, size_t smem,
+                       cudaStream_t s, const LayerArgs& a) {
+  const bool prof = h->prof && h->prof_used < kProfCapacity;
+  if (h->prof && !prof) h->prof_overflow = true;
+  if (prof) cudaEventRecord(h->prof_ev[2 * h->prof_used], s);
+  cudaError_t e = launch_pdl(k, grid, block, smem, s, a, h->ws);
+  if (prof && e == cudaSuccess) {
+    cudaEventRecord(h->prof_ev[2 * h->prof_used + 1], s);
+    h->prof_kind[h->prof_used++] = kind;
+  }
+  return e;
+}
+
+rtp_status enqueue_layer(rtp_handle* h, const LayerArgs& a, cudaStream_t s) {
+  const int slots = a.B * a.nret;
+  cudaError_t e;
+  if (a.nret > 0 && !a.dense) {
+    e = launch_one(h, 0, score_kernel, dim3(h->ws.n_score_chunks, slots), dim3(kSelThreads), 0,
+                   s, a);
+    if (e != cudaSuccess) return cuda_fail(e, "score_kernel launch");
+    e = launch_one(h, 1, hist_kernel, dim3(h->ws.n_sel_chunks, slots), dim3(kSelThreads), 0, s,
+                   a);
+    if (e != cudaSuccess) return cuda_fail(e, "hist_kernel launch");
+    e = launch_one(h, 2, compact_kernel, dim3(h->ws.n_sel_chunks, slots), dim3(kSelThreads), 0,
+                   s, a);
+    if (e != cudaSuccess) return cuda_fail(e, "compact_kernel launch");
+  }
+  e = launch_one(h, 3, attend_kernel, dim3(h->attend_grid), dim3(kAttendThreads), h->attend_smem,
+                 s, a);
+  if (e != cudaSuccess) return cuda_fail(e, "attend_kernel launch");
+  return RTP_OK;
+}
+
+struct DeviceGuard {
+  int prev = -1;
+  explicit DeviceGuard(int dev) {
+    if (cudaGetDevice(&prev) != cudaSuccess) prev = -1;
+    if (prev != dev) cudaSetDevice(dev);
+  }
+  ~DeviceGuard() {
+    int cur = -1;
+    if (prev >= 0 && cudaGetDevice(&cur) == cudaSuccess && cur != prev) cudaSetDevice(prev);
+  }
+};
+
+}  // namespace
+
+extern "C" {
+
+void rtp_config_default(rtp_config* c, int num_layers, int batch, int num_q_heads,
+                        int num_kv_heads, int max_ctx) {
+  if (!c) return;
+  c->num_layers = num_layers;
+  c->batch = batch;
+  c->num_q_heads = num_q_heads;
+  c->num_kv_heads = num_kv_heads;
+  c->head_dim = 128;
+  c->idx_dim = 16;
+  c->max_ctx = max_ctx;
+  c->window = 8192;
+  c->sinks = 4;
+  c->num_bins = 256;
+  c->idx_range = 16.0f;
+  c->idx_scale = 0.25f;
+  c->attn_scale = (float)(1.0 / std::sqrt(128.0));
+}
+
+size_t rtp_workspace_bytes(const rtp_config* cfg) {
+  if (check_config(cfg) != RTP_OK) return 0;
+  int dev = 0, sms = 148;
+  if (cudaGetDevice(&dev) == cudaSuccess)
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  return plan_workspace(cfg, sms).total;
+}
+
+rtp_status rtp_create(const rtp_config* cfg, int device, rtp_handle** out) {
+  if (!out) return fail(RTP_ERR_INVALID_ARG, "out is NULL");
+  *out = nullptr;
+  rtp_status st = check_config(cfg);
+  if (st != RTP_OK) return st;
+  int ndev = 0;
+  cudaError_t e = cudaGetDeviceCount(&ndev);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaGetDeviceCount");
+  if (device < 0 || device >= ndev)
+    return fail(RTP_ERR_INVALID_ARG, "device %d out of range (%d devices)", device, ndev);
+  DeviceGuard guard(device);
+
+  rtp_handle* h = new rtp_handle();
+  h->cfg = *cfg;
+  h->device = device;
+  h->G = cfg->num_q_heads / cfg->num_kv_heads;
+  cudaDeviceGetAttribute(&h->num_sms, cudaDevAttrMultiProcessorCount, device);
+  h->attend_grid = h->num_sms;  // one persistent CTA per SM
+
+  const WsPlan p = plan_workspace(cfg, h->attend_grid);
+  const size_t L = (size_t)cfg->num_layers, B = (size_t)cfg->batch;
+  const size_t q_bytes = L * B * cfg->num_q_heads * kHeadDim * 2;
+  const size_t qi_bytes = L * B * cfg->num_kv_heads * kIdxDim * 2;
+  const size_t out_bytes = L * B * cfg->num_q_heads * kHeadDim * 4;
+  const size_t stage_q_off = p.total;
+  const size_t stage_qi_off = round_up(stage_q_off + q_bytes, 256);
+  const size_t stage_seq_off = round_up(stage_qi_off + qi_bytes, 256);
+  const size_t stage_out_off = round_up(stage_seq_off + B * 4, 256);
+  h->ws_bytes = round_up(stage_out_off + out_bytes, 256);
+
+  e = cudaMalloc(&h->ws_mem, h->ws_bytes);
+  if (e != cudaSuccess) {
+    const size_t bytes = h->ws_bytes;
+    delete h;
+    cudaGetLastError();
+    return fail(RTP_ERR_OOM, "cudaMalloc of %zu workspace bytes failed", bytes);
+  }
+  e = cudaMemset(h->ws_mem, 0, h->ws_bytes);
+  if (e != cudaSuccess) {
+    cudaFree(h->ws_mem);
+    delete h;
+    return cuda_fail(e, "cudaMemset");
+  }
+  char* base = static_cast<char*>(h->ws_mem);
+  Workspace& w = h->ws;
+  w.scores = reinterpret_cast<float*>(base + p.off[0]);
+  w.chunk_max = reinterpret_cast<float*>(base + p.off[1]);
+  w.hist = reinterpret_cast<unsigned long long*>(base + p.off[2]);
+  w.s_max = reinterpret_cast<float*>(base + p.off[3]);
+  w.bstar = reinterpret_cast<int*>(base + p.off[4]);
+  w.mass_total = reinterpret_cast<unsigned long long*>(base + p.off[5]);
+  w.sel_idx = reinterpret_cast<int*>(base + p.off[6]);
+  w.chunk_cnt = reinterpret_cast<int*>(base + p.off[7]);
+  w.chunk_off = reinterpret_cast<int*>(base + p.off[8]);
+  w.sel_total = reinterpret_cast<int*>(base + p.off[9]);
+  w.sel_n = reinterpret_cast<int*>(base + p.off[10]);
+  w.ticket_hist = reinterpret_cast<unsigned*>(base + p.off[11]);
+  w.ticket_compact = reinterpret_cast<unsigned*>(base + p.off[12]);
+  w.ticket_attend = reinterpret_cast<unsigned*>(base + p.off[13]);
+  w.partials = reinterpret_cast<float*>(base + p.off[14]);
+  w.status = reinterpret_cast<unsigned*>(base + p.off[15]);
+  w.n_score_chunks = (cfg->max_ctx + kScoreChunk - 1) / kScoreChunk;
+  w.n_sel_chunks = (cfg->max_ctx + kSelChunk - 1) / kSelChunk;
+  h->stage_q = base + stage_q_off;
+  h->stage_qidx = base + stage_qi_off;
+  h->stage_seq = reinterpret_cast<int*>(base + stage_seq_off);
+  h->stage_out = reinterpret_cast<float*>(base + stage_out_off);
+
+  h->attend_smem = attend_smem_bytes(w.n_sel_chunks);
+  int max_optin = 0;
+  cudaDeviceGetAttribute(&max_optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, device);
+  if (h->attend_smem + 1024 > (size_t)max_optin) {
+    cudaFree(h->ws_mem);
+    delete h;
+    return fail(RTP_ERR_UNSUPPORTED, "max_ctx too large for the attention kernel's shared memory");
+  }
+  e = cudaFuncSetAttribute(attend_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           (int)h->attend_smem);
+  if (e != cudaSuccess) {
+    cudaFree(h->ws_mem);
+    delete h;
+    return cuda_fail(e, "cudaFuncSetAttribute(attend_kernel)");
+  }
+  *out = h;
+  return ok();
+}
+
+rtp_status rtp_destroy(rtp_handle* h) {
+  if (!h) return ok();
+  DeviceGuard guard(h->device);
+  cudaDeviceSynchronize();
+  for (cudaEvent_t ev : h->prof_ev) cudaEventDestroy(ev);
+  cudaError_t e = cudaFree(h->ws_mem);
+  delete h;
+  if (e != cudaSuccess) return cuda_fail(e, "cudaFree");
+  return ok();
+}
+
+rtp_status rtp_decode_step(rtp_handle* h, int layer, const rtp_layer_io* io, void* stream) {
+  if (!h) return fail(RTP_ERR_INVALID_ARG, "handle is NULL");
+  if (layer < 0 || layer >= h->cfg.num_layers)
+    return fail(RTP_ERR_INVALID_ARG, "layer %d outside [0, %d)", layer, h->cfg.num_layers);
+  if (!io) return fail(RTP_ERR_INVALID_ARG, "io is NULL");
+  if (!io->retrieval_mask) return fail(RTP_ERR_INVALID_ARG, "retrieval_mask is NULL");
+  LayerArgs a = make_args(h, io);
+  a.nret = 0;
+  for (int kvh = 0; kvh < a.Hkv; ++kvh) {
+    if (io->retrieval_mask[kvh]) {
+      a.slot_of_kvh[kvh] = (short)a.nret;
+      a.ret_kvh[a.nret++] = (short)kvh;
+    }
+  }
+  rtp_status st = check_io(h, io, a.nret > 0);
+  if (st != RTP_OK) return st;
+  DeviceGuard guard(h->device);
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  st = enqueue_layer(h, a, s);
+  if (st != RTP_OK) return st;
+  h->last_valid = true;
+  h->last_stream = s;
+  h->last_nret = a.nret;
+  memcpy(h->last_slot_of_kvh, a.slot_of_kvh, sizeof h->last_slot_of_kvh);
+  return ok();
+}
+
+rtp_status rtp_dense_decode(rtp_handle* h, const rtp_layer_io* io, void* stream) {
+  if (!h) return fail(RTP_ERR_INVALID_ARG, "handle is NULL");
+  rtp_status st = check_io(h, io, false);
+  if (st != RTP_OK) return st;
+  LayerArgs a = make_args(h, io);
+  a.dense = 1;
+  a.nret = 0;
+  DeviceGuard guard(h->device);
+  st = enqueue_layer(h, a, static_cast<cudaStream_t>(stream));
+  return st == RTP_OK ? ok() : st;
+}
+
+rtp_status rtp_decode_step_host(rtp_handle* h, int num_layers, const void* q_host,
+                                const void* q_idx_host, const int32_t* seq_lens_host,
+                                const void* const* k_cache, const void* const* v_cache,
+                                const void* const* k_idx, const uint8_t* masks, float top_p,
+                                float* out_host, void* stream) {
+  if (!h) return fail(RTP_ERR_INVALID_ARG, "handle is NULL");
+  if (num_layers < 1 || num_layers > h->cfg.num_layers)
+    return fail(RTP_ERR_INVALID_ARG, "num_layers outside [1, %d]", h->cfg.num_layers);
+  if (!q_host || !seq_lens_host || !k_cache || !v_cache || !masks || !out_host)
+    return fail(RTP_ERR_INVALID_ARG, "a required host pointer is NULL");
+  const rtp_config& c = h->cfg;
+  const size_t L = (size_t)num_layers, B = (size_t)c.batch;
+  const size_t q_layer = B * c.num_q_heads * kHeadDim;       // elements per layer
+  const size_t qi_layer = B * c.num_kv_heads * kIdxDim;
+  bool any_ret = false;
+  for (size_t i = 0; i < L * c.num_kv_heads; ++i) any_ret |= masks[i] != 0;
+  if (any_ret && (!q_idx_host || !k_idx))
+    return fail(RTP_ERR_INVALID_ARG, "q_idx_host and k_idx are required for retrieval heads");
+  for (int b = 0; b < c.batch; ++b)
+    if (seq_lens_host[b] < 1 || seq_lens_host[b] > c.max_ctx)
+      return fail(RTP_ERR_INVALID_ARG, "seq_lens_host[%d] = %d outside [1, %d]", b,
+                  seq_lens_host[b], c.max_ctx);
+  DeviceGuard guard(h->device);
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  cudaError_t e = cudaMemcpyAsync(h->stage_q, q_host, L * q_layer * 2, cudaMemcpyHostToDevice, s);
+  if (e == cudaSuccess && any_ret)
+    e = cudaMemcpyAsync(h->stage_qidx, q_idx_host, L * qi_layer * 2, cudaMemcpyHostToDevice, s);
+  if (e == cudaSuccess)
+    e = cudaMemcpyAsync(h->stage_seq, seq_lens_host, B * 4, cudaMemcpyHostToDevice, s);
+  if (e != cudaSuccess) return cuda_fail(e, "host-to-device copy");
+  for (int l = 0; l < num_layers; ++l) {
+    rtp_layer_io io;
+    memset(&io, 0, sizeof io);
+    io.q = static_cast<const char*>(h->stage_q) + (size_t)l * q_layer * 2;
+    io.q_idx = static_cast<const char*>(h->stage_qidx) + (size_t)l * qi_layer * 2;
+    io.k_cache = k_cache[l];
+    io.v_cache = v_cache[l];
+    io.k_idx = k_idx ? k_idx[l] : nullptr;
+    io.seq_lens = h->stage_seq;
+    io.retrieval_mask = masks + (size_t)l * c.num_kv_heads;
+    io.top_p = top_p;
+    io.out = h->stage_out + (size_t)l * q_layer;
+    rtp_status st = rtp_decode_step(h, l, &io, stream);
+    if (st != RTP_OK) return st;
+  }
+  e = cudaMemcpyAsync(out_host, h->stage_out, L * q_layer * 4, cudaMemcpyDeviceToHost, s);
+  if (e != cudaSuccess) return cuda_fail(e, "device-to-host copy");
+  e = cudaStreamSynchronize(s);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaStreamSynchronize");
+  return ok();
+}
+
+static rtp_status last_slot(rtp_handle* h, int b, int kvh, int* slot) {
+  if (!h) return fail(RTP_ERR_INVALID_ARG, "handle is NULL");
+  if (!h->last_valid) return fail(RTP_ERR_INVALID_ARG, "no rtp_decode_step on this handle yet");
+  if (b < 0 || b >= h->cfg.batch || kvh < 0 || kvh >= h->cfg.num_kv_heads)
+    return fail(RTP_ERR_INVALID_ARG, "(b, kvh) = (%d, %d) out of range", b, kvh);
+  const int j = h->last_slot_of_kvh[kvh];
+  if (j < 0) return fail(RTP_ERR_INVALID_ARG, "kv head %d was local in the last call", kvh);
+  *slot = b * h->last_nret + j;
+  return RTP_OK;
+}
+
+rtp_status rtp_get_selection(rtp_handle* h, int b, int kvh, int32_t* idx_out, int64_t cap,
+                             int64_t* count) {
+  int slot = 0;
+  rtp_status st = last_slot(h, b, kvh, &slot);
+  if (st != RTP_OK) return st;
+  if (!count) return fail(RTP_ERR_INVALID_ARG, "count is NULL");
+  if (cap > 0 && !idx_out) return fail(RTP_ERR_INVALID_ARG, "idx_out is NULL");
+  DeviceGuard guard(h->device);
+  cudaError_t e = cudaStreamSynchronize(h->last_stream);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaStreamSynchronize");
+  int total = 0, n = 0;
+  e = cudaMemcpy(&total, h->ws.sel_total + slot, 4, cudaMemcpyDeviceToHost);
+  if (e == cudaSuccess) e = cudaMemcpy(&n, h->ws.sel_n + slot, 4, cudaMemcpyDeviceToHost);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaMemcpy");
+  *count = total;
+  if (cap <= 0) return ok();
+  const int nch = (n + kSelChunk - 1) / kSelChunk;
+  std::vector<int> cnt(nch), sel((size_t)n);
+  e = cudaMemcpy(cnt.data(), h->ws.chunk_cnt + (size_t)slot * h->ws.n_sel_chunks, nch * 4,
+                 cudaMemcpyDeviceToHost);
+  if (e == cudaSuccess)
+    e = cudaMemcpy(sel.data(), h->ws.sel_idx + (size_t)slot * h->cfg.max_ctx, (size_t)n * 4,
+                   cudaMemcpyDeviceToHost);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaMemcpy");
+  int64_t k = 0;
+  for (int c = 0; c < nch && k < cap; ++c)
+    for (int i = 0; i < cnt[c] && k < cap; ++i) idx_out[k++] = sel[(size_t)c * kSelChunk + i];
+  return ok();
+}
+
+rtp_status rtp_get_threshold(rtp_handle* h, int b, int kvh, int* bstar, float* s_max) {
+  int slot = 0;
+  rtp_status st = last_slot(h, b, kvh, &slot);
+  if (st != RTP_OK) return st;
+  if (!bstar || !s_max) return fail(RTP_ERR_INVALID_ARG, "bstar and s_max must be non-NULL");
+  DeviceGuard guard(h->device);
+  cudaError_t e = cudaStreamSynchronize(h->last_stream);
+  if (e == cudaSuccess) e = cudaMemcpy(bstar, h->ws.bstar + slot, 4, cudaMemcpyDeviceToHost);
+  if (e == cudaSuccess) e = cudaMemcpy(s_max, h->ws.s_max + slot, 4, cudaMemcpyDeviceToHost);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaMemcpy");
+  return ok();
+}
+
+rtp_status rtp_get_device_status(rtp_handle* h, uint32_t* code) {
+  if (!h || !code) return fail(RTP_ERR_INVALID_ARG, "handle and code must be non-NULL");
+  DeviceGuard guard(h->device);
+  cudaError_t e = cudaDeviceSynchronize();
+  if (e == cudaSuccess) e = cudaMemcpy(code, h->ws.status, 4, cudaMemcpyDeviceToHost);
+  if (e == cudaSuccess) e = cudaMemset(h->ws.status, 0, 4);
+  if (e != cudaSuccess) return cuda_fail(e, "reading the device status");
+  if (*code) return fail(RTP_ERR_DEVICE_STATUS, "device status 0x%x", *code);
+  return ok();
+}
+
+rtp_status rtp_profile_enable(rtp_handle* h, int enable) {
+  if (!h) return fail(RTP_ERR_INVALID_ARG, "handle is NULL");
+  DeviceGuard guard(h->device);
+  if (enable && h->prof_ev.empty()) {
+    h->prof_ev.resize(2 * kProfCapacity);
+    h->prof_kind.resize(kProfCapacity);
+    for (auto& ev : h->prof_ev) {
+      cudaError_t e = cudaEventCreate(&ev);
+      if (e != cudaSuccess) return cuda_fail(e, "cudaEventCreate");
+    }
+  }
+  h->prof = enable != 0;
+  h->prof_used = 0;
+  h->prof_overflow = false;
+  return ok();
+}
+
+rtp_status rtp_profile_read(rtp_handle* h, double* ms, int64_t* launches) {
+  if (!h || !ms || !launches) return fail(RTP_ERR_INVALID_ARG, "NULL argument");
+  DeviceGuard guard(h->device);
+  for (int k = 0; k < 4; ++k) {
+    ms[k] = 0.0;
+    launches[k] = 0;
+  }
+  for (int i = 0; i < h->prof_used; ++i) {
+    float t = 0.f;
+    cudaError_t e = cudaEventSynchronize(h->prof_ev[2 * i + 1]);
+    if (e == cudaSuccess) e = cudaEventElapsedTime(&t, h->prof_ev[2 * i], h->prof_ev[2 * i + 1]);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaEventElapsedTime");
+    ms[h->prof_kind[i]] += t;
+    launches[h->prof_kind[i]] += 1;
+  }
+  const bool overflow = h->prof_overflow;
+  h->prof_used = 0;
+  h->prof_overflow = false;
+  if (overflow) return fail(RTP_ERR_INVALID_ARG, "profiling pool overflowed; read more often");
+  return ok();
+}
+
+const char* rtp_status_string(rtp_status s) {
+  switch (s) {
+    case RTP_OK: return "RTP_OK";
+    case RTP_ERR_INVALID_ARG: return "RTP_ERR_INVALID_ARG";
+    case RTP_ERR_UNSUPPORTED: return "RTP_ERR_UNSUPPORTED";
+    case RTP_ERR_OOM: return "RTP_ERR_OOM";
+    case RTP_ERR_CUDA: return "RTP_ERR_CUDA";
+    case RTP_ERR_DEVICE_STATUS: return "RTP_ERR_DEVICE_STATUS";
+  }
+  return "RTP_ERR_UNKNOWN";
+}
+
+const char* rtp_last_error(void) { return g_err; }
+
+}  // extern "C"

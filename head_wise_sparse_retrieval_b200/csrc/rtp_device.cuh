@@ -1,0 +1,179 @@
+// rtp_device.cuh -- device-side building blocks shared by the kernels of librtp (sm_100a).
+//
+// Inline PTX wrappers for: programmatic dependent launch, mbarriers with bounded waits,
+// 1-D bulk async copies (global -> shared, completed on an mbarrier), ldmatrix, movmatrix and
+// the warp-level bf16 MMA used to spare the FP32 pipes in the gather kernel.
+#pragma once
+
+#include <cstdint>
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+
+namespace rtp {
+
+constexpr int kHeadDim = 128;            // D
+constexpr int kIdxDim = 16;              // r
+constexpr int kBins = 256;               // histogram bins
+constexpr int kScoreChunk = 1024;        // tokens per indexer-score CTA
+constexpr int kSelChunk = 8192;          // tokens per histogram / compaction CTA
+constexpr int kSelThreads = 256;
+constexpr int kMaxGroup = 8;             // query heads per KV head handled by one MMA column set
+constexpr int kPartStride = 2 + kHeadDim;   // (m, l, o[128]) per query head in a partial
+constexpr double kFixedOne = 1099511627776.0;  // 2^40: fixed-point unit of histogram masses
+
+// Device status bits (mirrors include/rtp.h).
+constexpr unsigned kDevBadSeqlen = 0x1u;
+constexpr unsigned kDevWaitTimeout = 0x2u;
+constexpr unsigned kDevBadIndex = 0x4u;
+
+// Bounded waits give up after this long (ns of %globaltimer) and report kDevWaitTimeout.
+constexpr unsigned long long kWaitLimitNs = 2000000000ull;
+
+// ---- programmatic dependent launch ------------------------------------------------------
+
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_launch_dependents() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
+__device__ __forceinline__ unsigned long long global_ns() {
+  unsigned long long t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
+
+// ---- shared-memory addresses and mbarriers ------------------------------------------------
+
+__device__ __forceinline__ uint32_t smem_u32(const void* p) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+__device__ __forceinline__ void mbar_init(uint64_t* bar, unsigned count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count)
+               : "memory");
+}
+
+__device__ __forceinline__ void fence_mbar_init() {
+  asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+}
+
+__device__ __forceinline__ void fence_proxy_async_smem() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
+  asm volatile("{\n\t.reg .b64 st;\n\tmbarrier.arrive.shared::cta.b64 st, [%0];\n\t}" ::"r"(
+                   smem_u32(bar))
+               : "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* bar, unsigned bytes) {
+  asm volatile(
+      "{\n\t.reg .b64 st;\n\tmbarrier.arrive.expect_tx.shared::cta.b64 st, [%0], %1;\n\t}" ::"r"(
+          smem_u32(bar)),
+      "r"(bytes)
+      : "memory");
+}
+
+__device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, unsigned parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\tmbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
+// Waits for the phase of `parity` to complete. Gives up after kWaitLimitNs, sets
+// kDevWaitTimeout in *status and raises *abort_flag (shared) so that later waits of the CTA
+// return at once: control flow stays identical across warps and the kernel ends.
+__device__ __forceinline__ void mbar_wait_bounded(uint64_t* bar, unsigned parity,
+                                                  unsigned* status, volatile int* abort_flag) {
+  if (mbar_try_wait(bar, parity)) return;
+  const unsigned long long t0 = global_ns();
+  for (unsigned it = 0;; ++it) {
+    if (*abort_flag) return;
+    if (mbar_try_wait(bar, parity)) return;
+    if ((it & 255u) == 255u && global_ns() - t0 > kWaitLimitNs) {
+      atomicOr(status, kDevWaitTimeout);
+      *abort_flag = 1;
+      return;
+    }
+  }
+}
+
+// 1-D bulk copy global -> shared of `bytes` (multiple of 16, both addresses 16-byte aligned),
+// completing `bytes` of transaction count on `bar`. L2 policy: evict-first (read-once data).
+__device__ __forceinline__ void bulk_g2s(void* smem_dst, const void* gmem_src, unsigned bytes,
+                                         uint64_t* bar, uint64_t policy) {
+  asm volatile(
+      "cp.async.bulk.shared::cta.global.mbarrier::complete_tx::bytes.L2::cache_hint"
+      " [%0], [%1], %2, [%3], %4;" ::"r"(smem_u32(smem_dst)),
+      "l"(gmem_src), "r"(bytes), "r"(smem_u32(bar)), "l"(policy)
+      : "memory");
+}
+
+__device__ __forceinline__ uint64_t l2_policy_evict_first() {
+  uint64_t p;
+  asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(p));
+  return p;
+}
+
+__device__ __forceinline__ void named_barrier_sync(int id, int nthreads) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
+}
+
+// ---- warp-level matrix fragments ----------------------------------------------------------
+
+__device__ __forceinline__ void ldmatrix_x4(uint32_t (&r)[4], uint32_t addr) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+               : "r"(addr));
+}
+
+__device__ __forceinline__ void ldmatrix_x4_trans(uint32_t (&r)[4], uint32_t addr) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0,%1,%2,%3}, [%4];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+               : "r"(addr));
+}
+
+__device__ __forceinline__ uint32_t movmatrix_trans(uint32_t x) {
+  uint32_t y;
+  asm volatile("movmatrix.sync.aligned.m8n8.trans.b16 %0, %1;" : "=r"(y) : "r"(x));
+  return y;
+}
+
+// D = A(16x16, row) * B(16x8, col) + D, bf16 inputs, fp32 accumulators.
+__device__ __forceinline__ void mma_bf16_16816(float (&d)[4], const uint32_t (&a)[4],
+                                               uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
+      "{%8,%9}, {%0,%1,%2,%3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+
+__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
+  __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);  // .x = lo (low half), .y = hi
+  return *reinterpret_cast<uint32_t*>(&v);
+}
+
+__device__ __forceinline__ float bf16_lo(uint32_t v) { return __uint_as_float(v << 16); }
+__device__ __forceinline__ float bf16_hi(uint32_t v) { return __uint_as_float(v & 0xffff0000u); }
+
+// ---- the histogram bin of a scaled indexer score -------------------------------------------
+//
+// bin = clamp(256 + floor((s - s_max) * bin_scale), 0, 255), bin_scale = 256 / idx_range.
+// This equals floor((s - (s_max - idx_range)) * 256 / idx_range) clamped to [0, 255]. Every
+// kernel that bins a score calls this one function on the same fp32 inputs, so a token counted
+// in bin b by the histogram is selected by the compaction exactly when b >= b*.
+__device__ __forceinline__ int score_bin(float s, float s_max, float bin_scale) {
+  const float t = __fmul_rn(__fsub_rn(s, s_max), bin_scale);
+  const float f = floorf(t);                      // <= 0 for s <= s_max
+  const float c = fminf(fmaxf(f + 256.0f, 0.0f), 255.0f);
+  return static_cast<int>(c);
+}
+
+}  // namespace rtp

@@ -1,0 +1,186 @@
+/*
+ * rtp.h -- C-ABI of the B200 decode-step attention of RTPurbo (head-wise sparse retrieval).
+ *
+ * One call computes one layer of one decode step for a batch of sequences:
+ *
+ *   retrieval KV head (mask != 0), per sequence b with context N = seq_lens[b]:
+ *     s_n  = idx_scale * q_idx . k_idx[n]                       n < N      (indexer score)
+ *     bin  = clamp(floor((s_n - (s_max - idx_range)) * 256 / idx_range), 0, 255)
+ *     w_n  = exp(s_n - s_max);  M_b = sum_{bin(n)=b} w_n;  C_b = M_255 + ... + M_b
+ *     b*   = max{ b : C_b >= top_p * C_0 };  S = { n : bin(n) >= b* }  (sort-free top-p)
+ *     o_g  = sum_{n in S} softmax_S(attn_scale * q_g . k_n) v_n   for the G query heads g
+ *            of the KV head's GQA group (they share S)
+ *   local KV head (mask == 0):
+ *     the same o_g over T = {0 .. sinks-1} U {N-window .. N-1} (clipped to [0, N))
+ *
+ * Passages this follows (page title, then section / equation):
+ *   "Full Attention Strikes Back: Transferring Full Attention into Sparse within Hundred
+ *   Training Steps" (xllm-io paper review):
+ *     - section 三, 核心公式 / 自适应稀疏注意力: the low-rank indexer score s_h(m,n), taken
+ *       before RoPE, the sparse attention O_h(m) over S_h(m), and S_h(m) = Top-P(s_h, p);
+ *     - section 三, 硬件感知解码内核: sort-free top-p over a 256-bin histogram whose size does
+ *       not depend on the sequence length, scoring and selection fused;
+ *     - section 五, 测试配置: window 8192, 4 sink tokens, low-rank size 16, top-p 0.9.
+ *   "Technical Summary: Full Attention Strikes Back ..." (gist.science), Methodology 1 and 3:
+ *     local heads use a sliding window with attention sinks; retrieval heads select tokens
+ *     in decode by accumulating low-dimensional attention mass until p is reached.
+ *   The pages leave the bin edges, the indexer scale and the handling of GQA groups open;
+ *   the rules above are the readings this library implements.
+ *
+ * Conventions for every entry point:
+ *   - All tensors are row-major and contiguous. bf16 / fp16 tensors are passed as void*
+ *     (16-bit IEEE bfloat16 / binary16 values). Device pointers must be 16-byte aligned.
+ *   - The caller owns every buffer passed in. The handle owns only its workspace.
+ *   - Every call returns an rtp_status. Arguments are checked on the host before any
+ *     launch; on error nothing is enqueued. rtp_last_error() gives a one-line reason
+ *     (thread-local, valid until the next call on the same thread).
+ *   - Streams are cudaStream_t passed as void* (NULL = the legacy default stream).
+ *   - One handle serves one stream at a time: calls that overlap on the GPU through the
+ *     same handle race on its workspace.
+ */
+#ifndef RTP_H
+#define RTP_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define RTP_API __attribute__((visibility("default")))
+#else
+#define RTP_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    RTP_OK = 0,
+    RTP_ERR_INVALID_ARG = 1,   /* a NULL / misaligned pointer, a size out of range, ... */
+    RTP_ERR_UNSUPPORTED = 2,   /* a valid configuration this build does not implement    */
+    RTP_ERR_OOM = 3,           /* device workspace allocation failed (rtp_create only)   */
+    RTP_ERR_CUDA = 4,          /* a CUDA runtime call failed                             */
+    RTP_ERR_DEVICE_STATUS = 5  /* the kernels reported a problem (rtp_get_device_status) */
+} rtp_status;
+
+/* Device status bits, reported by rtp_get_device_status. */
+#define RTP_DEV_BAD_SEQLEN   0x1u  /* a seq_lens[b] outside [1, max_ctx]; it was clamped   */
+#define RTP_DEV_WAIT_TIMEOUT 0x2u  /* a bounded in-kernel wait gave up (output invalid)     */
+#define RTP_DEV_BAD_INDEX    0x4u  /* a token index outside [0, N) was about to be read     */
+
+typedef struct rtp_handle rtp_handle;
+
+typedef struct {
+    int num_layers;    /* layers of the model; rtp_decode_step's layer is checked against it   */
+    int batch;         /* B, >= 1                                                              */
+    int num_q_heads;   /* Hq; Hq % Hkv == 0                                                    */
+    int num_kv_heads;  /* Hkv, 1 .. 256; G = Hq / Hkv must be 1 .. 8                           */
+    int head_dim;      /* D, 128 only                                                          */
+    int idx_dim;       /* r, 16 only                                                           */
+    int max_ctx;       /* cache capacity per (b, KV head), 1 .. 2^28                           */
+    int window;        /* local-head sliding window, >= 1 (8192)                               */
+    int sinks;         /* local-head sink tokens, >= 0 (4)                                     */
+    int num_bins;      /* histogram bins, 256 only                                             */
+    float idx_range;   /* the bins cover [s_max - idx_range, s_max], > 0 (16)                  */
+    float idx_scale;   /* indexer score scale, > 0 (1/sqrt(16) = 0.25)                         */
+    float attn_scale;  /* attention logit scale, > 0 (1/sqrt(128))                            */
+} rtp_config;
+
+/* Fills *cfg with the pages' configuration for the given shape: head_dim 128, idx_dim 16,
+ * window 8192, sinks 4, 256 bins over a range of 16, idx_scale 0.25, attn_scale 1/sqrt(128). */
+RTP_API void rtp_config_default(rtp_config *cfg, int num_layers, int batch, int num_q_heads,
+                        int num_kv_heads, int max_ctx);
+
+/* Bytes of device workspace rtp_create allocates for cfg (0 if cfg is invalid). */
+RTP_API size_t rtp_workspace_bytes(const rtp_config *cfg);
+
+/* Creates a handle on CUDA device `device` and allocates its workspace, sized for the worst
+ * case (every KV head a retrieval head selecting all max_ctx tokens), so that no later call
+ * allocates. Errors: RTP_ERR_INVALID_ARG (bad cfg or out == NULL), RTP_ERR_UNSUPPORTED
+ * (head_dim, idx_dim, num_bins or G outside what is implemented), RTP_ERR_OOM, RTP_ERR_CUDA. */
+RTP_API rtp_status rtp_create(const rtp_config *cfg, int device, rtp_handle **out);
+
+/* Frees the workspace and the handle. NULL is accepted. Synchronises the device first. */
+RTP_API rtp_status rtp_destroy(rtp_handle *h);
+
+typedef struct {
+    const void *q;           /* bf16 [B][Hq][D], device: the current token's queries (RoPE'd)    */
+    const void *q_idx;       /* fp16 [B][Hkv][r], device: indexer queries W^Q q^pre; read for
+                                retrieval heads only (may be NULL when the mask has none)        */
+    const void *k_cache;     /* bf16 [B][Hkv][max_ctx][D], device: keys (RoPE'd)                 */
+    const void *v_cache;     /* bf16 [B][Hkv][max_ctx][D], device: values                        */
+    const void *k_idx;       /* fp16 [B][Hkv][max_ctx][r], device: indexer keys W^K k^pre; read
+                                for retrieval heads only (may be NULL when the mask has none)    */
+    const int32_t *seq_lens; /* [B], device: N_b, 1 <= N_b <= max_ctx. The caches already hold
+                                the current token at position N_b - 1.                          */
+    const uint8_t *retrieval_mask; /* [Hkv], HOST: nonzero marks a retrieval KV head           */
+    float top_p;             /* 0 < top_p <= 1                                                   */
+    float *out;              /* fp32 [B][Hq][D], device: attention output                        */
+    int32_t *sel_count;      /* optional [B][Hkv], device: receives |S| for retrieval heads and
+                                |T| for local heads; NULL to skip                                */
+} rtp_layer_io;
+
+/* Enqueues one layer of the decode step on `stream`. Asynchronous: no host synchronisation,
+ * no allocation, capturable in a CUDA graph (the mask is read on the host at call time and the
+ * launch shapes depend only on cfg and the mask). Errors (nothing enqueued): RTP_ERR_INVALID_ARG
+ * for a NULL handle / io / required pointer, a misaligned device pointer, top_p outside (0, 1]
+ * or layer outside [0, num_layers); RTP_ERR_CUDA if a launch fails. Problems only the device
+ * can see (seq_lens) are reported through rtp_get_device_status. */
+RTP_API rtp_status rtp_decode_step(rtp_handle *h, int layer, const rtp_layer_io *io, void *stream);
+
+/* Dense full attention over all N_b tokens for every KV head (top_p, q_idx, k_idx and the mask
+ * are ignored). The speedup denominator: same caches, same kernels, no selection. */
+RTP_API rtp_status rtp_dense_decode(rtp_handle *h, const rtp_layer_io *io, void *stream);
+
+/* Host-buffer variant of a whole decode step over `num_layers` layers: copies the queries
+ * q_host (bf16 [L][B][Hq][D]) and q_idx_host (fp16 [L][B][Hkv][r]) and seq_lens_host
+ * (int32 [B]) from host memory to the handle's device staging, runs rtp_decode_step for each
+ * layer l with the device caches k_cache[l], v_cache[l], k_idx[l] and the host mask
+ * masks[l * Hkv ...], and copies the fp32 outputs back into out_host ([L][B][Hq][D]).
+ * Host buffers should be pinned for the copies to be asynchronous. Synchronises `stream`
+ * before returning (the outputs are in out_host on return). Staging is allocated by
+ * rtp_create for cfg.num_layers layers. Errors as rtp_decode_step. */
+RTP_API rtp_status rtp_decode_step_host(rtp_handle *h, int num_layers, const void *q_host,
+                                const void *q_idx_host, const int32_t *seq_lens_host,
+                                const void *const *k_cache, const void *const *v_cache,
+                                const void *const *k_idx, const uint8_t *masks, float top_p,
+                                float *out_host, void *stream);
+
+/* Debug / parity: the ascending token positions selected for (b, kvh) by the most recent
+ * rtp_decode_step on this handle (which must have marked kvh as a retrieval head).
+ * Synchronises that call's stream. Writes min(cap, |S|) positions to idx_out (HOST) and |S| to
+ * *count. Errors: RTP_ERR_INVALID_ARG (no such head in the last call, NULL count). */
+RTP_API rtp_status rtp_get_selection(rtp_handle *h, int b, int kvh, int32_t *idx_out, int64_t cap,
+                             int64_t *count);
+
+/* Debug / parity: the threshold bin b* and the maximum indexer score s_max (fp32) the most
+ * recent rtp_decode_step used for (b, kvh). Synchronises that call's stream. */
+RTP_API rtp_status rtp_get_threshold(rtp_handle *h, int b, int kvh, int *bstar, float *s_max);
+
+/* Kernel profiling. While enabled, every kernel that rtp_decode_step / rtp_dense_decode
+ * launches on this handle is bracketed by two CUDA events recorded on the launch stream (the
+ * events are created here, so the decode calls still allocate nothing). Do not enable it while
+ * capturing a CUDA graph. Kernel classes: 0 indexer score, 1 histogram + threshold,
+ * 2 compaction, 3 attention. The event pool holds 1024 launches; rtp_profile_read empties it.
+ * Errors: RTP_ERR_CUDA if the events cannot be created. */
+RTP_API rtp_status rtp_profile_enable(rtp_handle *h, int enable);
+
+/* Synchronises the recorded launches, adds their durations (ms) and counts per kernel class
+ * into ms[4] and launches[4] (overwritten), and empties the pool. */
+RTP_API rtp_status rtp_profile_read(rtp_handle *h, double *ms, int64_t *launches);
+
+/* Reads and clears the device status word (RTP_DEV_* bits) after synchronising the device.
+ * Returns RTP_ERR_DEVICE_STATUS when a bit was set, RTP_OK otherwise. */
+RTP_API rtp_status rtp_get_device_status(rtp_handle *h, uint32_t *code);
+
+/* Static string for a status code. */
+RTP_API const char *rtp_status_string(rtp_status s);
+
+/* One-line reason for the last error returned on this thread ("" if none). */
+RTP_API const char *rtp_last_error(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* RTP_H */

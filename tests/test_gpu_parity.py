@@ -1,0 +1,236 @@
+"""Parity of the CUDA library (called through its C-ABI) with the fp64 oracle, on a B200."""
+import numpy as np
+import pytest
+import torch
+
+from head_wise_sparse_retrieval_b200 import rtp
+from head_wise_sparse_retrieval_b200 import workloads as W
+
+from parity_utils import (check_layer, check_output, make_handle, oracle_head, run_layer,
+                          MEAN_ABS)
+
+pytestmark = pytest.mark.gpu
+
+DEV = "cuda"
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _needs_gpu():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    rtp.load()
+
+
+def _run(plan, layer=0, top_p=None, heads=None, poison=False, exact=True, **cfg):
+    li = W.make_layer(plan, layer, DEV, poison_tail=poison)
+    with make_handle(plan, **cfg) as h:
+        rep = check_layer(h, plan, li, layer, top_p, heads, exact=exact)
+    return rep
+
+
+def test_tiny_selects_the_needles():
+    p = W.plan("tiny")
+    li = W.make_layer(p, 0, DEV)
+    with make_handle(p) as h:
+        rep = check_layer(h, p, li, 0)
+        sel = h.selection(0, 0)
+    assert sel.tolist() == li.needles[(0, 0)].tolist()
+    assert rep.heads[0]["sel"].n_gpu == 3
+
+
+@pytest.mark.parametrize("query", ["conc", "diffuse", "flat"])
+def test_one_layer(query):
+    p = W.plan("one_layer", query=query)
+    rep = _run(p)
+    r = rep.heads[0]["sel"]
+    if query == "conc":
+        assert r.n_gpu <= 16
+    if query == "diffuse":
+        assert 3000 < r.n_gpu < 30000
+    assert r.n_exact <= r.n_gpu
+
+
+def test_batch_decode_full_size():
+    p = W.plan("batch_decode")
+    rep = _run(p, exact=False)
+    assert len(rep.heads) == 32
+
+
+@pytest.mark.parametrize("seq_lens", [
+    [1, 2, 3, 4, 5, 17, 64, 65],
+    [4095, 4096, 4097, 8191, 8192, 8193, 8196, 8197],
+    [20000, 1, 12345, 8197, 16384, 16385, 3, 9000],
+])
+def test_ragged_lengths_and_poisoned_tail(seq_lens):
+    """Ragged contexts around tile, chunk and window boundaries; the cache beyond N is NaN so
+    any read past the context shows up in the output."""
+    B = len(seq_lens)
+    kinds = [[W.KIND_DIFFUSE, W.KIND_LOCAL, W.KIND_CONC, W.KIND_FLAT] for _ in range(B)]
+    needles = [[0, 0, 3, 0] for _ in range(B)]
+    p = W.custom(batch=B, num_q_heads=32, num_kv_heads=4, seq_lens=seq_lens,
+                 max_ctx=max(seq_lens) + 37, retrieval=[1, 0, 1, 1], kinds=kinds,
+                 n_needles=needles, seed=sum(seq_lens) % 1000)
+    _run(p, poison=True)
+
+
+@pytest.mark.parametrize("G", [1, 2, 4, 8])
+def test_group_sizes(G):
+    H = 3
+    p = W.custom(batch=2, num_q_heads=H * G, num_kv_heads=H, seq_lens=[9000, 3000],
+                 max_ctx=9001, retrieval=[1, 0, 1],
+                 kinds=[[W.KIND_DIFFUSE, 0, W.KIND_CONC]] * 2, n_needles=[[0, 0, 5]] * 2,
+                 seed=G)
+    _run(p)
+
+
+@pytest.mark.parametrize("top_p", [0.01, 0.5, 0.8, 0.95, 1.0])
+def test_top_p_values(top_p):
+    p = W.custom(batch=1, num_q_heads=16, num_kv_heads=2, seq_lens=[30000], max_ctx=30000,
+                 retrieval=[1, 1], kinds=[[W.KIND_DIFFUSE, W.KIND_FLAT]], seed=7)
+    rep = _run(p, top_p=top_p)
+    if top_p == 1.0:
+        assert all(h["sel"].n_gpu == 30000 for h in rep.heads)
+
+
+def test_small_window_and_no_sinks():
+    p = W.custom(batch=2, num_q_heads=16, num_kv_heads=2, seq_lens=[5000, 100], max_ctx=5000,
+                 retrieval=[0, 0], kinds=[[0, 0]] * 2, seed=9, window=777, sinks=0)
+    _run(p, window=777, sinks=0)
+
+
+def test_all_retrieval_heads():
+    p = W.custom(batch=2, num_q_heads=32, num_kv_heads=4, seq_lens=[40000, 25000],
+                 max_ctx=40000, retrieval=[1, 1, 1, 1],
+                 kinds=[[W.KIND_CONC, W.KIND_DIFFUSE, W.KIND_FLAT, W.KIND_CONC]] * 2,
+                 n_needles=[[1, 0, 0, 64]] * 2, seed=11)
+    _run(p)
+
+
+def test_dense_decode_matches_oracle():
+    p = W.custom(batch=2, num_q_heads=32, num_kv_heads=4, seq_lens=[33000, 7],
+                 max_ctx=33000, retrieval=[1, 0, 0, 0],
+                 kinds=[[W.KIND_CONC, 0, 0, 0]] * 2, n_needles=[[3, 0, 0, 0]] * 2, seed=12)
+    li = W.make_layer(p, 0, DEV)
+    with make_handle(p) as h:
+        out, _ = run_layer(h, p, li, 0, dense=True)
+    out = out.cpu().numpy()
+    for b in range(2):
+        for kvh in range(4):
+            ho = oracle_head(li, b, kvh, False, 0.9, 8, dense=True)
+            check_output(out[b, kvh * 8:(kvh + 1) * 8], ho.out, f"dense b{b} kvh{kvh}")
+
+
+def test_p_one_equals_dense():
+    p = W.custom(batch=1, num_q_heads=16, num_kv_heads=2, seq_lens=[20000], max_ctx=20000,
+                 retrieval=[1, 1], kinds=[[W.KIND_CONC, W.KIND_DIFFUSE]],
+                 n_needles=[[4, 0]], seed=13)
+    li = W.make_layer(p, 0, DEV)
+    with make_handle(p) as h:
+        sparse, cnt = run_layer(h, p, li, 0, top_p=1.0)
+        dense, _ = run_layer(h, p, li, 0, dense=True)
+    assert cnt.cpu().tolist() == [[20000, 20000]]
+    assert torch.equal(sparse, dense)
+
+
+def test_deterministic_reruns():
+    p = W.plan("one_layer", query="diffuse")
+    li = W.make_layer(p, 0, DEV)
+    with make_handle(p) as h:
+        o1, c1 = run_layer(h, p, li, 0)
+        s1 = h.selection(0, 0)
+        o2, c2 = run_layer(h, p, li, 0)
+        s2 = h.selection(0, 0)
+    assert torch.equal(o1, o2) and torch.equal(c1, c2) and np.array_equal(s1, s2)
+
+
+def test_cuda_graph_replay_matches_eager():
+    p = W.plan("one_layer", query="conc")
+    li = W.make_layer(p, 0, DEV)
+    L = rtp.layer_from(li)
+    with make_handle(p) as h:
+        eager, _ = run_layer(h, p, li, 0)
+        out = torch.zeros_like(eager)
+        s = torch.cuda.Stream()
+        s.wait_stream(torch.cuda.current_stream())
+        with torch.cuda.stream(s):
+            h.decode_step(0, L, p.retrieval[0], p.top_p, out, stream=s)
+        torch.cuda.current_stream().wait_stream(s)
+        torch.cuda.synchronize()
+        g = torch.cuda.CUDAGraph()
+        out.zero_()
+        with torch.cuda.graph(g):
+            h.decode_step(0, L, p.retrieval[0], p.top_p, out)
+        out.zero_()
+        g.replay()
+        torch.cuda.synchronize()
+        assert torch.equal(out, eager)
+        del g
+
+
+def test_host_buffer_entry_matches_device_entry():
+    p = W.plan("long_context", num_layers=2, ctx=20000)
+    lis = [W.make_layer(p, l, DEV) for l in range(2)]
+    with make_handle(p) as h:
+        dev_out = [run_layer(h, p, li, l)[0] for l, li in enumerate(lis)]
+        q = torch.stack([li.q for li in lis]).cpu().pin_memory()
+        qi = torch.stack([li.q_idx for li in lis]).cpu().pin_memory()
+        seq = lis[0].seq_lens.cpu().pin_memory()
+        out = torch.empty((2,) + tuple(dev_out[0].shape), dtype=torch.float32).pin_memory()
+        h.decode_step_host(q, qi, seq, [rtp.layer_from(li) for li in lis], p.retrieval,
+                           p.top_p, out)
+    for l in range(2):
+        assert torch.equal(out[l], dev_out[l].cpu())
+
+
+def test_bad_seq_len_is_reported_not_faulted():
+    p = W.custom(batch=2, num_q_heads=8, num_kv_heads=1, seq_lens=[100, 50], max_ctx=128,
+                 retrieval=[1], kinds=[[W.KIND_CONC]] * 2, n_needles=[[2]] * 2, seed=14)
+    li = W.make_layer(p, 0, DEV)
+    li.seq_lens[1] = 1000  # beyond max_ctx: clamped on the device, reported in the status word
+    with make_handle(p) as h:
+        out, _ = run_layer(h, p, li, 0)
+        code = h.device_status()
+        assert code & rtp.DEV_BAD_SEQLEN
+        assert h.device_status() == 0  # reading clears it
+    assert torch.isfinite(out[0]).all()
+
+
+def test_host_side_argument_errors():
+    p = W.plan("tiny")
+    li = W.make_layer(p, 0, DEV)
+    with make_handle(p) as h:
+        out = torch.empty((1, 8, 128), dtype=torch.float32, device=DEV)
+        L = rtp.layer_from(li)
+        with pytest.raises(rtp.RtpError) as e:
+            h.decode_step(0, L, [1], 0.0, out)
+        assert e.value.status == rtp.RTP_ERR_INVALID_ARG
+        with pytest.raises(rtp.RtpError):
+            h.decode_step(0, L, [1], 1.5, out)
+        with pytest.raises(rtp.RtpError):
+            h.decode_step(1, L, [1], 0.9, out)  # layer out of range
+        bad = rtp.Layer(li.q, li.q_idx, li.k_cache.view(-1)[1:], li.v_cache, li.k_idx, li.seq_lens)
+        with pytest.raises(rtp.RtpError):
+            h.decode_step(0, bad, [1], 0.9, out)  # misaligned cache pointer
+        with pytest.raises(rtp.RtpError):
+            h.selection(0, 0)  # no successful decode_step yet
+
+
+@pytest.mark.slow
+@pytest.mark.parametrize("name", ["long_context", "ctx_1m"])
+def test_long_configs_sampled_layers(name):
+    """Full-size layers of the 48-layer workloads, in the launch configuration the benchmark
+    times (one call per layer, same handle configuration); every head of the sampled layers is
+    compared with the oracle."""
+    p = W.plan(name)
+    # a layer with a conc retrieval head, one with a diffuse/flat one, one with none
+    conc = [l for l in range(48) if (p.kind[l] == W.KIND_CONC).any()]
+    other = [l for l in range(48) if ((p.kind[l] == W.KIND_DIFFUSE) |
+                                      (p.kind[l] == W.KIND_FLAT)).any()]
+    none = [l for l in range(48) if not p.retrieval[l].any()]
+    layers = [conc[0], other[0], none[0]]
+    with make_handle(p) as h:
+        for l in layers:
+            li = W.make_layer(p, l, DEV)
+            check_layer(h, p, li, l, exact=False)
+            del li
+            torch.cuda.empty_cache()
