@@ -289,8 +289,9 @@ def main():
     g = torch.cuda.CUDAGraph()
     with torch.cuda.graph(g, stream=stream):
         step()
-    for _ in range(args.warmup):
-        g.replay()
+    with torch.cuda.stream(stream):  # a graph replays on the current stream
+        for _ in range(args.warmup):
+            g.replay()
     torch.cuda.synchronize()
 
     sampler = ClockSampler(dev.index if world == 1 else local)
@@ -302,10 +303,11 @@ def main():
     if world > 1:
         dist.barrier()
     torch.cuda.synchronize()
-    e0.record(stream)
-    for _ in range(args.steps):
-        g.replay()
-    e1.record(stream)
+    with torch.cuda.stream(stream):
+        e0.record(stream)
+        for _ in range(args.steps):
+            g.replay()
+        e1.record(stream)
     torch.cuda.synchronize()
     if world > 1:
         dist.barrier()
@@ -341,16 +343,18 @@ def main():
         gd = torch.cuda.CUDAGraph()
         with torch.cuda.graph(gd, stream=stream):
             step(dense=True)
-        for _ in range(3):
-            gd.replay()
+        with torch.cuda.stream(stream):
+            for _ in range(3):
+                gd.replay()
         torch.cuda.synchronize()
         nd = max(3, min(args.steps, 5))
         d0 = torch.cuda.Event(enable_timing=True)
         d1 = torch.cuda.Event(enable_timing=True)
-        d0.record(stream)
-        for _ in range(nd):
-            gd.replay()
-        d1.record(stream)
+        with torch.cuda.stream(stream):
+            d0.record(stream)
+            for _ in range(nd):
+                gd.replay()
+            d1.record(stream)
         torch.cuda.synchronize()
         dms = d0.elapsed_time(d1) / nd
         dense_bytes = sum(int(plan.seq_lens[b]) * ROW_BYTES for b in range(B)) * Hkv * L

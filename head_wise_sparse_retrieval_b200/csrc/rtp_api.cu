@@ -102,9 +102,10 @@ struct WsPlan {
 // Byte offsets of the workspace arrays (each 256-byte aligned).
 WsPlan plan_workspace(const rtp_config* c, int attend_grid) {
   const size_t slots = (size_t)c->batch * c->num_kv_heads;
-  const size_t nmax = (size_t)c->max_ctx;
+  const size_t nmax = round_up((size_t)c->max_ctx, 64);  // per-slot stride (16-byte loads)
   const size_t nsc = (nmax + kScoreChunk - 1) / kScoreChunk;
   const size_t nsel = (nmax + kSelChunk - 1) / kSelChunk;
+  const size_t ngroups = ((size_t)attend_grid + kMergeFanIn - 1) / kMergeFanIn;
   const size_t sizes[] = {
       slots * nmax * 4,                      // 0 scores
       slots * nsc * 4,                       // 1 chunk_max
@@ -113,15 +114,17 @@ WsPlan plan_workspace(const rtp_config* c, int attend_grid) {
       slots * 4,                             // 4 bstar
       slots * 8,                             // 5 mass_total
       slots * nmax * 4,                      // 6 sel_idx
-      slots * nsel * 4,                      // 7 chunk_cnt
+      slots * nsel * kBins * 4,              // 7 chunk_bins
       slots * (nsel + 1) * 4,                // 8 chunk_off
       slots * 4,                             // 9 sel_total
       slots * 4,                             // 10 sel_n
       slots * 4,                             // 11 ticket_hist
-      slots * 4,                             // 12 ticket_compact
+      4,                                     // 12 (unused)
       slots * 4,                             // 13 ticket_attend
-      ((size_t)attend_grid + slots) * kMaxGroup * kPartStride * 4,  // 14 partials
+      ((size_t)attend_grid + slots) * kPartFloats * 4,  // 14 partials
       256,                                   // 15 status
+      slots * ngroups * 4,                   // 16 ticket_group
+      slots * ngroups * kPartFloats * 4,  // 17 group_partials
   };
   WsPlan p{};
   size_t at = 0;
@@ -292,7 +295,8 @@ rtp_status rtp_create(const rtp_config* cfg, int device, rtp_handle** out) {
   h->device = device;
   h->G = cfg->num_q_heads / cfg->num_kv_heads;
   cudaDeviceGetAttribute(&h->num_sms, cudaDevAttrMultiProcessorCount, device);
-  h->attend_grid = h->num_sms;  // one persistent CTA per SM
+  h->attend_grid = h->num_sms * kAttendCtasPerSm;  // persistent: every CTA resident
+  if (h->attend_grid > 2 * kMergeFanIn * kMergeFanIn) h->attend_grid = 2 * kMergeFanIn * kMergeFanIn;
 
   const WsPlan p = plan_workspace(cfg, h->attend_grid);
   const size_t L = (size_t)cfg->num_layers, B = (size_t)cfg->batch;
@@ -327,15 +331,18 @@ rtp_status rtp_create(const rtp_config* cfg, int device, rtp_handle** out) {
   w.bstar = reinterpret_cast<int*>(base + p.off[4]);
   w.mass_total = reinterpret_cast<unsigned long long*>(base + p.off[5]);
   w.sel_idx = reinterpret_cast<int*>(base + p.off[6]);
-  w.chunk_cnt = reinterpret_cast<int*>(base + p.off[7]);
+  w.chunk_bins = reinterpret_cast<uint32_t*>(base + p.off[7]);
   w.chunk_off = reinterpret_cast<int*>(base + p.off[8]);
   w.sel_total = reinterpret_cast<int*>(base + p.off[9]);
   w.sel_n = reinterpret_cast<int*>(base + p.off[10]);
   w.ticket_hist = reinterpret_cast<unsigned*>(base + p.off[11]);
-  w.ticket_compact = reinterpret_cast<unsigned*>(base + p.off[12]);
   w.ticket_attend = reinterpret_cast<unsigned*>(base + p.off[13]);
   w.partials = reinterpret_cast<float*>(base + p.off[14]);
   w.status = reinterpret_cast<unsigned*>(base + p.off[15]);
+  w.ticket_group = reinterpret_cast<unsigned*>(base + p.off[16]);
+  w.group_partials = reinterpret_cast<float*>(base + p.off[17]);
+  w.n_merge_groups = (h->attend_grid + kMergeFanIn - 1) / kMergeFanIn;
+  w.ld = (int)round_up((size_t)cfg->max_ctx, 64);
   w.n_score_chunks = (cfg->max_ctx + kScoreChunk - 1) / kScoreChunk;
   w.n_sel_chunks = (cfg->max_ctx + kSelChunk - 1) / kSelChunk;
   h->stage_q = base + stage_q_off;
@@ -343,16 +350,18 @@ rtp_status rtp_create(const rtp_config* cfg, int device, rtp_handle** out) {
   h->stage_seq = reinterpret_cast<int*>(base + stage_seq_off);
   h->stage_out = reinterpret_cast<float*>(base + stage_out_off);
 
-  h->attend_smem = attend_smem_bytes(w.n_sel_chunks);
+  h->attend_smem = attend_smem_bytes(cfg->batch * cfg->num_kv_heads, cfg->batch);
   int max_optin = 0;
   cudaDeviceGetAttribute(&max_optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, device);
-  if (h->attend_smem + 1024 > (size_t)max_optin) {
+  if (h->attend_smem + 4096 > (size_t)max_optin / kAttendCtasPerSm) {
     cudaFree(h->ws_mem);
     delete h;
     return fail(RTP_ERR_UNSUPPORTED, "max_ctx too large for the attention kernel's shared memory");
   }
   e = cudaFuncSetAttribute(attend_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            (int)h->attend_smem);
+  if (e == cudaSuccess)
+    e = cudaFuncSetAttribute(attend_kernel, cudaFuncAttributePreferredSharedMemoryCarveout, 100);
   if (e != cudaSuccess) {
     cudaFree(h->ws_mem);
     delete h;
@@ -491,17 +500,11 @@ rtp_status rtp_get_selection(rtp_handle* h, int b, int kvh, int32_t* idx_out, in
   if (e != cudaSuccess) return cuda_fail(e, "cudaMemcpy");
   *count = total;
   if (cap <= 0) return ok();
-  const int nch = (n + kSelChunk - 1) / kSelChunk;
-  std::vector<int> cnt(nch), sel((size_t)n);
-  e = cudaMemcpy(cnt.data(), h->ws.chunk_cnt + (size_t)slot * h->ws.n_sel_chunks, nch * 4,
+  const int64_t k = total < cap ? total : cap;
+  e = cudaMemcpy(idx_out, h->ws.sel_idx + (size_t)slot * h->ws.ld, (size_t)k * 4,
                  cudaMemcpyDeviceToHost);
-  if (e == cudaSuccess)
-    e = cudaMemcpy(sel.data(), h->ws.sel_idx + (size_t)slot * h->cfg.max_ctx, (size_t)n * 4,
-                   cudaMemcpyDeviceToHost);
   if (e != cudaSuccess) return cuda_fail(e, "cudaMemcpy");
-  int64_t k = 0;
-  for (int c = 0; c < nch && k < cap; ++c)
-    for (int i = 0; i < cnt[c] && k < cap; ++i) idx_out[k++] = sel[(size_t)c * kSelChunk + i];
+  (void)n;
   return ok();
 }
 

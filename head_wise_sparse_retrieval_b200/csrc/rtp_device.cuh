@@ -1,8 +1,8 @@
 // rtp_device.cuh -- device-side building blocks shared by the kernels of librtp (sm_100a).
 //
 // Inline PTX wrappers for: programmatic dependent launch, mbarriers with bounded waits,
-// 1-D bulk async copies (global -> shared, completed on an mbarrier), ldmatrix, movmatrix and
-// the warp-level bf16 MMA used to spare the FP32 pipes in the gather kernel.
+// asynchronous copies global -> shared (cp.async, 1-D bulk), ldmatrix, movmatrix and the
+// warp-level bf16 MMA used to spare the FP32 pipes in the gather kernel.
 #pragma once
 
 #include <cstdint>
@@ -15,10 +15,13 @@ constexpr int kHeadDim = 128;            // D
 constexpr int kIdxDim = 16;              // r
 constexpr int kBins = 256;               // histogram bins
 constexpr int kScoreChunk = 1024;        // tokens per indexer-score CTA
-constexpr int kSelChunk = 8192;          // tokens per histogram / compaction CTA
 constexpr int kSelThreads = 256;
+constexpr int kPerThread = 16;           // consecutive tokens per thread in hist / compaction
+constexpr int kSelChunk = kSelThreads * kPerThread;  // tokens per hist / compaction CTA (4096)
 constexpr int kMaxGroup = 8;             // query heads per KV head handled by one MMA column set
-constexpr int kPartStride = 2 + kHeadDim;   // (m, l, o[128]) per query head in a partial
+// a partial of one KV head's attention: o[8][128] (unnormalised), then m[8] (log2 domain), l[8]
+constexpr int kPartO = kMaxGroup * kHeadDim;
+constexpr int kPartFloats = kPartO + 2 * kMaxGroup;
 constexpr double kFixedOne = 1099511627776.0;  // 2^40: fixed-point unit of histogram masses
 
 // Device status bits (mirrors include/rtp.h).
@@ -119,6 +122,22 @@ __device__ __forceinline__ uint64_t l2_policy_evict_first() {
   uint64_t p;
   asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(p));
   return p;
+}
+
+// 16-byte asynchronous copy global -> shared (L2 only, evict-first). src_bytes = 0 reads
+// nothing and fills the 16 bytes with zeros (ragged tiles).
+__device__ __forceinline__ void cp_async_16(uint32_t smem_dst, const void* gmem_src,
+                                            unsigned src_bytes, uint64_t policy) {
+  asm volatile("cp.async.cg.shared.global.L2::cache_hint [%0], [%1], 16, %2, %3;" ::"r"(smem_dst),
+               "l"(gmem_src), "r"(src_bytes), "l"(policy)
+               : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() {
+  asm volatile("cp.async.commit_group;" ::: "memory");
+}
+template <int N>
+__device__ __forceinline__ void cp_async_wait() {
+  asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
 }
 
 __device__ __forceinline__ void named_barrier_sync(int id, int nthreads) {

@@ -13,24 +13,27 @@ constexpr int kMaxKvHeads = 256;
 // Device workspace owned by a handle. Slot = b * nret + j for the j-th retrieval KV head of
 // the current layer (the workspace is sized for nret = Hkv).
 struct Workspace {
-  float* scores;                  // [slots][max_ctx]        scaled indexer scores
+  float* scores;                  // [slots][ld]             scaled indexer scores
   float* chunk_max;               // [slots][n_score_chunks] per-CTA maxima of the scores
   unsigned long long* hist;       // [slots][256]            fixed-point (2^-40) bin masses
   float* s_max;                   // [slots]
   int* bstar;                     // [slots]
   unsigned long long* mass_total; // [slots]                 C_0 in fixed point
-  int* sel_idx;                   // [slots][max_ctx]        selected positions, per 8192-chunk
-  int* chunk_cnt;                 // [slots][n_sel_chunks]   selected per chunk
-  int* chunk_off;                 // [slots][n_sel_chunks+1] exclusive prefix of chunk_cnt
+  int* sel_idx;                   // [slots][ld]             selected positions, ascending
+  uint32_t* chunk_bins;           // [slots][n_sel_chunks][256] tokens per bin and chunk
+  int* chunk_off;                 // [slots][n_sel_chunks+1] selected tokens before each chunk
   int* sel_total;                 // [slots]                 |S|
   int* sel_n;                     // [slots]                 N the selection was made over
   unsigned* ticket_hist;          // [slots]
-  unsigned* ticket_compact;       // [slots]
-  unsigned* ticket_attend;        // [B*Hkv]
-  float* partials;                // [(attend_ctas + B*Hkv)][8][2 + 128]
+  unsigned* ticket_attend;        // [B*Hkv]                 merge of a head's groups
+  unsigned* ticket_group;         // [B*Hkv][n_merge_groups] merge of a group's pieces
+  float* partials;                // [(attend_ctas + B*Hkv)][kPartFloats]  one per piece
+  float* group_partials;          // [B*Hkv][n_merge_groups][kPartFloats]
   unsigned* status;               // [1] RTP_DEV_* bits
+  int ld;                         // per-slot stride of scores / sel_idx: max_ctx rounded up to 64
   int n_score_chunks;             // ceil(max_ctx / kScoreChunk)
   int n_sel_chunks;               // ceil(max_ctx / kSelChunk)
+  int n_merge_groups;             // ceil(attend_ctas / kMergeFanIn)
 };
 
 struct LayerArgs {
@@ -55,14 +58,15 @@ __global__ void hist_kernel(const LayerArgs a, const Workspace w);
 __global__ void compact_kernel(const LayerArgs a, const Workspace w);
 __global__ void attend_kernel(const LayerArgs a, const Workspace w);
 
-constexpr int kAttendConsumerWarps = 4;
-constexpr int kAttendThreads = (kAttendConsumerWarps + 1) * 32;
-constexpr int kAttendTile = 16 * kAttendConsumerWarps;   // tokens per pipeline stage
-constexpr int kAttendStages = 4;
-constexpr int kRowBytes = 128 * 2;                       // one K or V row in HBM
-constexpr int kRowPitch = kRowBytes + 16;                // padded row in shared memory
+constexpr int kAttendWarps = 4;                          // warps per attention CTA
+constexpr int kAttendDepth = 3;                          // cp.async stages per warp
+constexpr int kAttendCtasPerSm = 2;                      // resident attention CTAs per SM
+constexpr int kAttendThreads = kAttendWarps * 32;
+constexpr int kRowBytes = 128 * 2;                       // one K or V row
 constexpr int kMaxAttendHeads = 1024;                    // B * Hkv per layer
+constexpr int kMergeFanIn = 16;                          // pieces merged per tree node
+// the attention grid is at most kMergeFanIn * 2 * kMergeFanIn CTAs (two merge levels)
 
-size_t attend_smem_bytes(int n_sel_chunks);
+size_t attend_smem_bytes(int nheads, int batch);
 
 }  // namespace rtp

@@ -10,12 +10,14 @@
 //                  a lane pair per token), writes the fp32 scaled scores (they stay in L2)
 //                  and one maximum per 1024-token chunk;
 //   hist_kernel    s_max = max of the chunk maxima; bins every score relative to s_max and
-//                  adds exp(s - s_max) to a shared 256-bin histogram in 2^-40 fixed point
+//                  adds exp(s - s_max) to 256 shared bins in 2^-40 fixed point
 //                  (integer adds: the result does not depend on the order of arrival); the
 //                  last CTA of a slot (atomic ticket, no waiting) scans the bins from the top
 //                  with one warp and writes b*;
-//   compact_kernel re-bins with the same function and emits the selected positions of each
-//                  8192-token chunk in ascending order; the last CTA writes the chunk offsets.
+//                  The same CTAs count tokens per bin and chunk, so once b* is known the last
+//                  CTA also writes how many tokens each chunk selects and their prefix;
+//   compact_kernel re-bins with the same function and writes the selected positions, in
+//                  ascending order, into one dense list (each chunk at its prefix offset).
 // Bins need the global s_max, so the scores make one round trip through L2 (4 B per token
 // against 32 B of indexer keys read from HBM).
 #include "rtp_device.cuh"
@@ -57,10 +59,7 @@ __global__ void __launch_bounds__(kSelThreads) score_kernel(const LayerArgs a, c
 
   if (blockIdx.x == 0) {  // reset what the next two kernels accumulate into
     w.hist[(size_t)slot * kBins + threadIdx.x] = 0ull;
-    if (threadIdx.x == 0) {
-      w.ticket_hist[slot] = 0u;
-      w.ticket_compact[slot] = 0u;
-    }
+    if (threadIdx.x == 0) w.ticket_hist[slot] = 0u;
   }
   pdl_launch_dependents();
 
@@ -83,7 +82,7 @@ __global__ void __launch_bounds__(kSelThreads) score_kernel(const LayerArgs a, c
     }
   }
   const uint4* keys = reinterpret_cast<const uint4*>(a.k_idx + head * (size_t)a.max_ctx * kIdxDim);
-  float* sc = w.scores + (size_t)slot * a.max_ctx;
+  float* sc = w.scores + (size_t)slot * w.ld;
 
   constexpr int kIter = kScoreChunk / (kSelThreads / 2);  // 8 tokens per lane pair
   uint4 kv[kIter];
@@ -119,13 +118,65 @@ __global__ void __launch_bounds__(kSelThreads) score_kernel(const LayerArgs a, c
   if (threadIdx.x == 0) w.chunk_max[(size_t)slot * w.n_score_chunks + blockIdx.x] = mx;
 }
 
-// ---- 2. mass histogram + threshold bin ---------------------------------------------------
+// ---- 2. mass histogram + threshold bin + chunk offsets ------------------------------------
+
+// Block-wide exclusive scan of one int per thread (256 threads); returns the block total.
+__device__ __forceinline__ int block_excl_scan_256(int v, int& excl, int* warp_tot) {
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  int x = v;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int y = __shfl_up_sync(0xffffffffu, x, o);
+    if (lane >= o) x += y;
+  }
+  if (lane == 31) warp_tot[warp] = x;
+  __syncthreads();
+  int before = 0, all = 0;
+#pragma unroll
+  for (int k = 0; k < kSelThreads / 32; ++k) {
+    const int t = warp_tot[k];
+    before += (k < warp) ? t : 0;
+    all += t;
+  }
+  __syncthreads();
+  excl = before + x - v;
+  return all;
+}
+
+// Loads the kPerThread consecutive scores of this thread (positions n..n+kPerThread-1), with
+// -inf past n1.
+__device__ __forceinline__ void load_scores(const float* sc, int n, int n1, float (&v)[kPerThread]) {
+  if (n + kPerThread <= n1) {
+#pragma unroll
+    for (int k = 0; k < kPerThread; k += 4) {
+      const float4 f = __ldcg(reinterpret_cast<const float4*>(sc + n + k));
+      v[k] = f.x;
+      v[k + 1] = f.y;
+      v[k + 2] = f.z;
+      v[k + 3] = f.w;
+    }
+  } else {
+#pragma unroll
+    for (int k = 0; k < kPerThread; ++k) v[k] = (n + k < n1) ? __ldcg(sc + n + k) : -INFINITY;
+  }
+}
 
 __global__ void __launch_bounds__(kSelThreads) hist_kernel(const LayerArgs a, const Workspace w) {
-  __shared__ unsigned long long hist[kBins];
-  __shared__ float red[kSelThreads / 32];
-  __shared__ int is_last;
-  hist[threadIdx.x] = 0ull;  // before the dependency wait: overlaps the previous kernel
+  // Per-warp histograms of the 2^-40 fixed-point masses, split into 32-bit low and high words
+  // (native shared-memory atomics; the carry of the low word is detected from the returned old
+  // value), and one token-count histogram. Integer sums: exact, independent of arrival order.
+  constexpr int kWarps = kSelThreads / 32;
+  __shared__ uint32_t wlo[kWarps][kBins];
+  __shared__ uint32_t whi[kWarps][kBins];
+  __shared__ uint32_t cnt[kBins];
+  __shared__ float red[kWarps];
+  __shared__ int warp_tot[kWarps];
+  __shared__ int is_last, bstar_s, carry_s;
+  for (int i = threadIdx.x; i < kWarps * kBins; i += kSelThreads) {
+    (&wlo[0][0])[i] = 0u;  // before the dependency wait: overlaps the previous kernel
+    (&whi[0][0])[i] = 0u;
+  }
+  cnt[threadIdx.x] = 0u;
   pdl_wait();
   pdl_launch_dependents();
 
@@ -135,154 +186,110 @@ __global__ void __launch_bounds__(kSelThreads) hist_kernel(const LayerArgs a, co
   const int n0 = blockIdx.x * kSelChunk;
   if (n0 >= N) return;
   const int n1 = min(n0 + kSelChunk, N);
+  const int warp = threadIdx.x >> 5;
 
   // s_max over the chunk maxima of the whole context (max is order-independent)
   const int nsc = (N + kScoreChunk - 1) / kScoreChunk;
   float m = -INFINITY;
   for (int i = threadIdx.x; i < nsc; i += kSelThreads)
     m = fmaxf(m, __ldcg(w.chunk_max + (size_t)slot * w.n_score_chunks + i));
-  const float s_max = block_max_256(m, red);  // also orders the hist[] reset before the adds
+  const float s_max = block_max_256(m, red);  // also orders the zero fill before the adds
 
-  const float* sc = w.scores + (size_t)slot * a.max_ctx;
-  for (int n = n0 + threadIdx.x; n < n1; n += kSelThreads) {
-    const float s = __ldcg(sc + n);
+  const float* sc = w.scores + (size_t)slot * w.ld;
+  float sv[kPerThread];
+  load_scores(sc, n0 + threadIdx.x * kPerThread, n1, sv);
+  uint32_t* lo_h = wlo[warp];
+  uint32_t* hi_h = whi[warp];
+#pragma unroll
+  for (int k = 0; k < kPerThread; ++k) {
+    const float s = sv[k];
+    if (s == -INFINITY) continue;
     const int bin = score_bin(s, s_max, a.bin_scale);
     const float wgt = expf(s - s_max);                       // in (0, 1]
     const unsigned long long fx = __float2ull_rn(wgt * 1099511627776.0f);  // * 2^40, exact
-    if (fx) atomicAdd(&hist[bin], fx);
+    const uint32_t lo = (uint32_t)fx;
+    uint32_t hi = (uint32_t)(fx >> 32);
+    if (lo) {
+      const uint32_t old = atomicAdd(lo_h + bin, lo);
+      hi += (old + lo < old) ? 1u : 0u;                      // carry out of the low word
+    }
+    if (hi) atomicAdd(hi_h + bin, hi);
+    atomicAdd(cnt + bin, 1u);
   }
   __syncthreads();
   {
-    const unsigned long long v = hist[threadIdx.x];
+    unsigned long long v = 0ull;
+#pragma unroll
+    for (int k = 0; k < kWarps; ++k)
+      v += ((unsigned long long)whi[k][threadIdx.x] << 32) + wlo[k][threadIdx.x];
     if (v) atomicAdd(w.hist + (size_t)slot * kBins + threadIdx.x, v);
+    w.chunk_bins[((size_t)slot * w.n_sel_chunks + blockIdx.x) * kBins + threadIdx.x] =
+        cnt[threadIdx.x];
   }
   __threadfence();
   __syncthreads();
   if (threadIdx.x == 0) {
     const unsigned nhc = (unsigned)((N + kSelChunk - 1) / kSelChunk);
     is_last = (atomicAdd(w.ticket_hist + slot, 1u) == nhc - 1u);
-  }
-  __syncthreads();
-  if (!is_last || threadIdx.x >= 32) return;
-
-  // last CTA of this slot: one warp, 8 bins per lane, suffix sums from the top bin down
-  __threadfence();
-  const int lane = threadIdx.x;
-  unsigned long long v[8], lane_sum = 0ull;
-#pragma unroll
-  for (int i = 0; i < 8; ++i) {
-    v[i] = __ldcg(w.hist + (size_t)slot * kBins + lane * 8 + i);
-    lane_sum += v[i];
-  }
-  unsigned long long incl = lane_sum;  // sum over lanes >= lane
-#pragma unroll
-  for (int o = 1; o < 32; o <<= 1) {
-    const unsigned long long y = __shfl_down_sync(0xffffffffu, incl, o);
-    if (lane + o < 32) incl += y;
-  }
-  const unsigned long long total = __shfl_sync(0xffffffffu, incl, 0);
-  const double target = (double)a.top_p * (double)total;
-  unsigned long long c = incl - lane_sum;  // mass of the bins above this lane's
-  int best = -1;
-#pragma unroll
-  for (int i = 7; i >= 0; --i) {
-    c += v[i];
-    if (best < 0 && (double)c >= target) best = lane * 8 + i;
-  }
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) best = max(best, __shfl_xor_sync(0xffffffffu, best, o));
-  if (lane == 0) {
-    w.bstar[slot] = best < 0 ? 0 : best;
-    w.s_max[slot] = s_max;
-    w.mass_total[slot] = total;
-    w.ticket_hist[slot] = 0u;
-  }
-}
-
-// ---- 3. ordered compaction of the selected positions --------------------------------------
-
-__global__ void __launch_bounds__(kSelThreads) compact_kernel(const LayerArgs a,
-                                                              const Workspace w) {
-  __shared__ int warp_cnt[kSelThreads / 32];
-  __shared__ int is_last;
-  __shared__ int carry_s;
-  pdl_wait();
-  pdl_launch_dependents();
-
-  const int slot = blockIdx.y;
-  const int b = slot / a.nret, kvh = a.ret_kvh[slot % a.nret];
-  const int N = clamp_seq_len(a, b, w.status, false);
-  const int n0 = blockIdx.x * kSelChunk;
-  if (n0 >= N) return;
-  const int n1 = min(n0 + kSelChunk, N);
-  const int bstar = __ldcg(w.bstar + slot);
-  const float s_max = __ldcg(w.s_max + slot);
-  const float* sc = w.scores + (size_t)slot * a.max_ctx;
-  int* out = w.sel_idx + (size_t)slot * a.max_ctx + n0;  // chunk c writes from position n0
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const unsigned lt_mask = (1u << lane) - 1u;
-
-  constexpr int kBatch = 8;
-  int running = 0;
-  for (int base = n0; base < n1; base += kBatch * kSelThreads) {
-    bool flag[kBatch];
-#pragma unroll
-    for (int k = 0; k < kBatch; ++k) {
-      const int n = base + k * kSelThreads + threadIdx.x;
-      flag[k] = (n < n1) && score_bin(__ldcg(sc + n), s_max, a.bin_scale) >= bstar;
-    }
-#pragma unroll
-    for (int k = 0; k < kBatch; ++k) {
-      const unsigned ballot = __ballot_sync(0xffffffffu, flag[k]);
-      if (lane == 0) warp_cnt[warp] = __popc(ballot);
-      __syncthreads();
-      int before = 0, all = 0;
-#pragma unroll
-      for (int i = 0; i < kSelThreads / 32; ++i) {
-        const int c = warp_cnt[i];
-        before += (i < warp) ? c : 0;
-        all += c;
-      }
-      if (flag[k]) out[running + before + __popc(ballot & lt_mask)] = base + k * kSelThreads + threadIdx.x;
-      running += all;
-      __syncthreads();
-    }
-  }
-  if (threadIdx.x == 0) w.chunk_cnt[(size_t)slot * w.n_sel_chunks + blockIdx.x] = running;
-  __threadfence();
-  __syncthreads();
-  if (threadIdx.x == 0) {
-    const unsigned nch = (unsigned)((N + kSelChunk - 1) / kSelChunk);
-    is_last = (atomicAdd(w.ticket_compact + slot, 1u) == nch - 1u);
     carry_s = 0;
   }
   __syncthreads();
   if (!is_last) return;
-
-  // last CTA: exclusive prefix of the per-chunk counts
   __threadfence();
-  const int nch = (N + kSelChunk - 1) / kSelChunk;
-  const int* cnt = w.chunk_cnt + (size_t)slot * w.n_sel_chunks;
-  int* off = w.chunk_off + (size_t)slot * (w.n_sel_chunks + 1);
-  for (int base = 0; base < nch; base += kSelThreads) {
-    const int i = base + threadIdx.x;
-    const int v = (i < nch) ? __ldcg(cnt + i) : 0;
-    int x = v;  // inclusive warp scan
+
+  // ---- last CTA of this slot: b* by one warp (8 bins per lane, suffix sums from the top) ----
+  if (threadIdx.x < 32) {
+    const int lane = threadIdx.x;
+    unsigned long long v[8], lane_sum = 0ull;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      v[i] = __ldcg(w.hist + (size_t)slot * kBins + lane * 8 + i);
+      lane_sum += v[i];
+    }
+    unsigned long long incl = lane_sum;  // sum over lanes >= lane
 #pragma unroll
     for (int o = 1; o < 32; o <<= 1) {
-      const int y = __shfl_up_sync(0xffffffffu, x, o);
-      if (lane >= o) x += y;
+      const unsigned long long y = __shfl_down_sync(0xffffffffu, incl, o);
+      if (lane + o < 32) incl += y;
     }
-    if (lane == 31) warp_cnt[warp] = x;
-    __syncthreads();
-    int before = 0, all = 0;
+    const unsigned long long total = __shfl_sync(0xffffffffu, incl, 0);
+    const double target = (double)a.top_p * (double)total;
+    unsigned long long c = incl - lane_sum;  // mass of the bins above this lane's
+    int best = -1;
 #pragma unroll
-    for (int k = 0; k < kSelThreads / 32; ++k) {
-      before += (k < warp) ? warp_cnt[k] : 0;
-      all += warp_cnt[k];
+    for (int i = 7; i >= 0; --i) {
+      c += v[i];
+      if (best < 0 && (double)c >= target) best = lane * 8 + i;
     }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) best = max(best, __shfl_xor_sync(0xffffffffu, best, o));
+    if (lane == 0) {
+      bstar_s = best < 0 ? 0 : best;
+      w.mass_total[slot] = total;
+    }
+  }
+  __syncthreads();
+  const int bs = bstar_s;
+
+  // ---- selected tokens per chunk (bins >= b*) and their exclusive prefix ----
+  const int nch = (N + kSelChunk - 1) / kSelChunk;
+  int* off = w.chunk_off + (size_t)slot * (w.n_sel_chunks + 1);
+  for (int base = 0; base < nch; base += kSelThreads) {
+    const int cc = base + threadIdx.x;
+    int v = 0;
+    if (cc < nch) {
+      const uint32_t* row = w.chunk_bins + ((size_t)slot * w.n_sel_chunks + cc) * kBins;
+      int bb = bs;
+      for (; bb < kBins && (bb & 3); ++bb) v += (int)__ldcg(row + bb);
+      for (; bb < kBins; bb += 4) {
+        const uint4 q = __ldcg(reinterpret_cast<const uint4*>(row + bb));
+        v += (int)(q.x + q.y + q.z + q.w);
+      }
+    }
+    int excl;
+    const int all = block_excl_scan_256(v, excl, warp_tot);
     const int carry = carry_s;
-    if (i < nch) off[i] = carry + before + x - v;
+    if (cc < nch) off[cc] = carry + excl;
     __syncthreads();
     if (threadIdx.x == 0) carry_s = carry + all;
     __syncthreads();
@@ -290,11 +297,47 @@ __global__ void __launch_bounds__(kSelThreads) compact_kernel(const LayerArgs a,
   if (threadIdx.x == 0) {
     const int total = carry_s;
     off[nch] = total;
+    w.bstar[slot] = bs;
+    w.s_max[slot] = s_max;
     w.sel_total[slot] = total;
     w.sel_n[slot] = N;
-    w.ticket_compact[slot] = 0u;
-    (void)kvh;
+    w.ticket_hist[slot] = 0u;
   }
+}
+
+// ---- 3. compaction: the selected positions, ascending, into one dense list -----------------
+
+__global__ void __launch_bounds__(kSelThreads) compact_kernel(const LayerArgs a,
+                                                              const Workspace w) {
+  __shared__ int warp_tot[kSelThreads / 32];
+  pdl_wait();
+  pdl_launch_dependents();
+
+  const int slot = blockIdx.y;
+  const int b = slot / a.nret;
+  const int N = clamp_seq_len(a, b, w.status, false);
+  const int n0 = blockIdx.x * kSelChunk;
+  if (n0 >= N) return;
+  const int n1 = min(n0 + kSelChunk, N);
+  const int bstar = __ldcg(w.bstar + slot);
+  const float s_max = __ldcg(w.s_max + slot);
+  const int base = __ldcg(w.chunk_off + (size_t)slot * (w.n_sel_chunks + 1) + blockIdx.x);
+  const float* sc = w.scores + (size_t)slot * w.ld;
+  int* out = w.sel_idx + (size_t)slot * w.ld;
+
+  const int n = n0 + threadIdx.x * kPerThread;  // this thread's kPerThread consecutive tokens
+  float sv[kPerThread];
+  load_scores(sc, n, n1, sv);
+  unsigned flags = 0u;
+#pragma unroll
+  for (int k = 0; k < kPerThread; ++k)
+    if (sv[k] != -INFINITY && score_bin(sv[k], s_max, a.bin_scale) >= bstar) flags |= 1u << k;
+  int excl;
+  block_excl_scan_256(__popc(flags), excl, warp_tot);
+  int at = base + excl;
+#pragma unroll
+  for (int k = 0; k < kPerThread; ++k)
+    if (flags & (1u << k)) out[at++] = n + k;
 }
 
 }  // namespace rtp
