@@ -283,7 +283,7 @@ def main():
         raise SystemExit(f"device status 0x{status:x} after the eager step")
     sel = [c.cpu().numpy() for c in cnts]
     total_bytes, attend_bytes, idx_bytes = step_bytes(plan, sel)
-    launches_per_step = sum(4 if plan.retrieval[l].any() else 1 for l in range(L))
+    launches_per_step = sum(2 if plan.retrieval[l].any() else 1 for l in range(L))
 
     # capture the whole step as one CUDA graph
     g = torch.cuda.CUDAGraph()
@@ -331,7 +331,7 @@ def main():
             acc[k][1] += n
     h.profile(False)
     kern = {k: {"ms_total_per_step": v[0] / prof_steps, "launches_per_step": v[1] / prof_steps}
-            for k, v in acc.items()}
+            for k, v in acc.items() if v[1]}
     att_ms = acc["attend"][0] / max(acc["attend"][1], 1)
     att_bytes_per_launch = attend_bytes / L
     hbm, peak_kind = _peaks()

@@ -279,9 +279,12 @@ __global__ void __launch_bounds__(kAttendThreads, kAttendCtasPerSm) attend_kerne
     const int b = hd / a.Hkv, kvh = hd - b * a.Hkv;
     const int N = sSeq[b];
     int len;
-    if (a.dense) {
+    const bool ret = !a.dense && a.slot_of_kvh[kvh] >= 0;
+    if ((a.heads == kHeadsLocal && ret) || (a.heads == kHeadsRetrieval && !ret)) {
+      len = 0;  // another launch of this layer covers the head
+    } else if (a.dense) {
       len = N;
-    } else if (a.slot_of_kvh[kvh] >= 0) {
+    } else if (ret) {
       len = __ldcg(w.sel_total + b * a.nret + a.slot_of_kvh[kvh]);
       len = len < 1 ? 1 : (len > N ? N : len);
     } else {
@@ -311,7 +314,7 @@ __global__ void __launch_bounds__(kAttendThreads, kAttendCtasPerSm) attend_kerne
   // P = min(grid, T) CTAs take part, so every range is non-empty and the pieces of a head are
   // exactly the CTAs c_first..c_last (the ticket count of its merge)
   const long long T = sOff[nheads];
-  const long long P = min((long long)gridDim.x, T);
+  const long long P = min((long long)gridDim.x, T);  // T >= 1: the launch covers >= 1 head
   if ((long long)blockIdx.x >= P) return;
   const long long t0 = (long long)blockIdx.x * T / P;
   const long long t1 = ((long long)blockIdx.x + 1) * T / P;

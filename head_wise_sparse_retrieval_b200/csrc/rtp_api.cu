@@ -17,6 +17,8 @@ struct rtp_handle {
   int num_sms = 0;
   int G = 0;
   int attend_grid = 0;
+  int select_grid = 0;
+  size_t select_smem = 0;
   size_t attend_smem = 0;
   void* ws_mem = nullptr;
   size_t ws_bytes = 0;
@@ -100,25 +102,23 @@ struct WsPlan {
 };
 
 // Byte offsets of the workspace arrays (each 256-byte aligned).
-WsPlan plan_workspace(const rtp_config* c, int attend_grid) {
+WsPlan plan_workspace(const rtp_config* c, int attend_grid, int select_grid) {
   const size_t slots = (size_t)c->batch * c->num_kv_heads;
   const size_t nmax = round_up((size_t)c->max_ctx, 64);  // per-slot stride (16-byte loads)
-  const size_t nsc = (nmax + kScoreChunk - 1) / kScoreChunk;
-  const size_t nsel = (nmax + kSelChunk - 1) / kSelChunk;
   const size_t ngroups = ((size_t)attend_grid + kMergeFanIn - 1) / kMergeFanIn;
   const size_t sizes[] = {
       slots * nmax * 4,                      // 0 scores
-      slots * nsc * 4,                       // 1 chunk_max
+      slots * (size_t)select_grid * 4,       // 1 cta_max
       slots * kBins * 8,                     // 2 hist
       slots * 4,                             // 3 s_max
       slots * 4,                             // 4 bstar
       slots * 8,                             // 5 mass_total
       slots * nmax * 4,                      // 6 sel_idx
-      slots * nsel * kBins * 4,              // 7 chunk_bins
-      slots * (nsel + 1) * 4,                // 8 chunk_off
+      slots * (size_t)select_grid * kBins * 4,  // 7 cta_bins
+      4,                                     // 8 (unused)
       slots * 4,                             // 9 sel_total
       slots * 4,                             // 10 sel_n
-      slots * 4,                             // 11 ticket_hist
+      (size_t)(2 + (4 * kMaxAttendHeads + 15) / 16) * 4,  // 11 grid_bar
       4,                                     // 12 (unused)
       slots * 4,                             // 13 ticket_attend
       ((size_t)attend_grid + slots) * kPartFloats * 4,  // 14 partials
@@ -138,17 +138,19 @@ WsPlan plan_workspace(const rtp_config* c, int attend_grid) {
 
 template <typename Kernel>
 cudaError_t launch_pdl(Kernel k, dim3 grid, dim3 block, size_t smem, cudaStream_t s,
-                       const LayerArgs& a, const Workspace& w) {
+                       const LayerArgs& a, const Workspace& w, bool cooperative) {
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = grid;
   cfg.blockDim = block;
   cfg.dynamicSmemBytes = smem;
   cfg.stream = s;
-  cudaLaunchAttribute attr[1];
+  cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
   attr[0].val.programmaticStreamSerializationAllowed = 1;
+  attr[1].id = cudaLaunchAttributeCooperative;
+  attr[1].val.cooperative = 1;
   cfg.attrs = attr;
-  cfg.numAttrs = 1;
+  cfg.numAttrs = cooperative ? 2 : 1;
   return cudaLaunchKernelEx(&cfg, k, a, w);
 }
 
@@ -204,11 +206,12 @@ constexpr int kProfCapacity = 1024;
 // Launches one kernel, bracketed by profiling events when the handle has profiling enabled.
 template <typename Kernel>
 cudaError_t launch_one(rtp_handle* h, int kind, Kernel k, dim3 grid, dim3 block, size_t smem,
-                       cudaStream_t s, const LayerArgs& a) {
+                       cudaStream_t s, const LayerArgs& a, const Workspace& ws,
+                       bool cooperative = false) {
   const bool prof = h->prof && h->prof_used < kProfCapacity;
   if (h->prof && !prof) h->prof_overflow = true;
   if (prof) cudaEventRecord(h->prof_ev[2 * h->prof_used], s);
-  cudaError_t e = launch_pdl(k, grid, block, smem, s, a, h->ws);
+  cudaError_t e = launch_pdl(k, grid, block, smem, s, a, ws, cooperative);
   if (prof && e == cudaSuccess) {
     cudaEventRecord(h->prof_ev[2 * h->prof_used + 1], s);
     h->prof_kind[h->prof_used++] = kind;
@@ -216,24 +219,18 @@ cudaError_t launch_one(rtp_handle* h, int kind, Kernel k, dim3 grid, dim3 block,
   return e;
 }
 
-rtp_status enqueue_layer(rtp_handle* h, const LayerArgs& a, cudaStream_t s) {
-  const int slots = a.B * a.nret;
+rtp_status enqueue_layer(rtp_handle* h, const LayerArgs& a0, cudaStream_t s) {
   cudaError_t e;
-  if (a.nret > 0 && !a.dense) {
-    e = launch_one(h, 0, score_kernel, dim3(h->ws.n_score_chunks, slots), dim3(kSelThreads), 0,
-                   s, a);
-    if (e != cudaSuccess) return cuda_fail(e, "score_kernel launch");
-    e = launch_one(h, 1, hist_kernel, dim3(h->ws.n_sel_chunks, slots), dim3(kSelThreads), 0, s,
-                   a);
-    if (e != cudaSuccess) return cuda_fail(e, "hist_kernel launch");
-    e = launch_one(h, 2, compact_kernel, dim3(h->ws.n_sel_chunks, slots), dim3(kSelThreads), 0,
-                   s, a);
-    if (e != cudaSuccess) return cuda_fail(e, "compact_kernel launch");
+  if (!a0.dense && a0.nret > 0) {
+    e = launch_one(h, 0, select_kernel, dim3(h->select_grid), dim3(kSelThreads), h->select_smem,
+                   s, a0, h->ws, true);
+    if (e != cudaSuccess) return cuda_fail(e, "select_kernel launch");
   }
-  e = launch_one(h, 3, attend_kernel, dim3(h->attend_grid), dim3(kAttendThreads), h->attend_smem,
-                 s, a);
-  if (e != cudaSuccess) return cuda_fail(e, "attend_kernel launch");
-  return RTP_OK;
+  LayerArgs a = a0;
+  a.heads = kHeadsAll;
+  e = launch_one(h, 1, attend_kernel, dim3(h->attend_grid), dim3(kAttendThreads), h->attend_smem,
+                 s, a, h->ws);
+  return e == cudaSuccess ? RTP_OK : cuda_fail(e, "attend_kernel launch");
 }
 
 struct DeviceGuard {
@@ -275,7 +272,7 @@ size_t rtp_workspace_bytes(const rtp_config* cfg) {
   int dev = 0, sms = 148;
   if (cudaGetDevice(&dev) == cudaSuccess)
     cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-  return plan_workspace(cfg, sms).total;
+  return plan_workspace(cfg, sms * kAttendCtasPerSm, sms * kMaxSelectCtasPerSm).total;
 }
 
 rtp_status rtp_create(const rtp_config* cfg, int device, rtp_handle** out) {
@@ -298,7 +295,21 @@ rtp_status rtp_create(const rtp_config* cfg, int device, rtp_handle** out) {
   h->attend_grid = h->num_sms * kAttendCtasPerSm;  // persistent: every CTA resident
   if (h->attend_grid > 2 * kMergeFanIn * kMergeFanIn) h->attend_grid = 2 * kMergeFanIn * kMergeFanIn;
 
-  const WsPlan p = plan_workspace(cfg, h->attend_grid);
+  h->select_smem = select_smem_bytes(cfg->batch * cfg->num_kv_heads);
+  e = cudaFuncSetAttribute(select_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           (int)h->select_smem);
+  int sel_per_sm = 0;
+  if (e == cudaSuccess)
+    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&sel_per_sm, select_kernel, kSelThreads,
+                                                      h->select_smem);
+  if (e != cudaSuccess || sel_per_sm < 1) {
+    delete h;
+    return e != cudaSuccess ? cuda_fail(e, "occupancy of select_kernel")
+                            : fail(RTP_ERR_UNSUPPORTED, "select_kernel does not fit an SM");
+  }
+  if (sel_per_sm > kMaxSelectCtasPerSm) sel_per_sm = kMaxSelectCtasPerSm;
+  h->select_grid = h->num_sms * sel_per_sm;  // cooperative: every CTA resident at once
+  const WsPlan p = plan_workspace(cfg, h->attend_grid, h->select_grid);
   const size_t L = (size_t)cfg->num_layers, B = (size_t)cfg->batch;
   const size_t q_bytes = L * B * cfg->num_q_heads * kHeadDim * 2;
   const size_t qi_bytes = L * B * cfg->num_kv_heads * kIdxDim * 2;
@@ -325,17 +336,16 @@ rtp_status rtp_create(const rtp_config* cfg, int device, rtp_handle** out) {
   char* base = static_cast<char*>(h->ws_mem);
   Workspace& w = h->ws;
   w.scores = reinterpret_cast<float*>(base + p.off[0]);
-  w.chunk_max = reinterpret_cast<float*>(base + p.off[1]);
+  w.cta_max = reinterpret_cast<float*>(base + p.off[1]);
   w.hist = reinterpret_cast<unsigned long long*>(base + p.off[2]);
   w.s_max = reinterpret_cast<float*>(base + p.off[3]);
   w.bstar = reinterpret_cast<int*>(base + p.off[4]);
   w.mass_total = reinterpret_cast<unsigned long long*>(base + p.off[5]);
   w.sel_idx = reinterpret_cast<int*>(base + p.off[6]);
-  w.chunk_bins = reinterpret_cast<uint32_t*>(base + p.off[7]);
-  w.chunk_off = reinterpret_cast<int*>(base + p.off[8]);
+  w.cta_bins = reinterpret_cast<uint32_t*>(base + p.off[7]);
   w.sel_total = reinterpret_cast<int*>(base + p.off[9]);
   w.sel_n = reinterpret_cast<int*>(base + p.off[10]);
-  w.ticket_hist = reinterpret_cast<unsigned*>(base + p.off[11]);
+  w.grid_bar = reinterpret_cast<unsigned*>(base + p.off[11]);
   w.ticket_attend = reinterpret_cast<unsigned*>(base + p.off[13]);
   w.partials = reinterpret_cast<float*>(base + p.off[14]);
   w.status = reinterpret_cast<unsigned*>(base + p.off[15]);
@@ -343,8 +353,6 @@ rtp_status rtp_create(const rtp_config* cfg, int device, rtp_handle** out) {
   w.group_partials = reinterpret_cast<float*>(base + p.off[17]);
   w.n_merge_groups = (h->attend_grid + kMergeFanIn - 1) / kMergeFanIn;
   w.ld = (int)round_up((size_t)cfg->max_ctx, 64);
-  w.n_score_chunks = (cfg->max_ctx + kScoreChunk - 1) / kScoreChunk;
-  w.n_sel_chunks = (cfg->max_ctx + kSelChunk - 1) / kSelChunk;
   h->stage_q = base + stage_q_off;
   h->stage_qidx = base + stage_qi_off;
   h->stage_seq = reinterpret_cast<int*>(base + stage_seq_off);
@@ -376,6 +384,7 @@ rtp_status rtp_destroy(rtp_handle* h) {
   DeviceGuard guard(h->device);
   cudaDeviceSynchronize();
   for (cudaEvent_t ev : h->prof_ev) cudaEventDestroy(ev);
+
   cudaError_t e = cudaFree(h->ws_mem);
   delete h;
   if (e != cudaSuccess) return cuda_fail(e, "cudaFree");

@@ -14,10 +14,8 @@ namespace rtp {
 constexpr int kHeadDim = 128;            // D
 constexpr int kIdxDim = 16;              // r
 constexpr int kBins = 256;               // histogram bins
-constexpr int kScoreChunk = 1024;        // tokens per indexer-score CTA
 constexpr int kSelThreads = 256;
-constexpr int kPerThread = 16;           // consecutive tokens per thread in hist / compaction
-constexpr int kSelChunk = kSelThreads * kPerThread;  // tokens per hist / compaction CTA (4096)
+constexpr int kPerThread = 16;           // consecutive tokens per thread in the compaction
 constexpr int kMaxGroup = 8;             // query heads per KV head handled by one MMA column set
 // a partial of one KV head's attention: o[8][128] (unnormalised), then m[8] (log2 domain), l[8]
 constexpr int kPartO = kMaxGroup * kHeadDim;
@@ -37,6 +35,12 @@ constexpr unsigned long long kWaitLimitNs = 2000000000ull;
 __device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
 __device__ __forceinline__ void pdl_launch_dependents() {
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
+__device__ __forceinline__ unsigned ld_acquire_gpu(const unsigned* p) {
+  unsigned v;
+  asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
 }
 
 __device__ __forceinline__ unsigned long long global_ns() {

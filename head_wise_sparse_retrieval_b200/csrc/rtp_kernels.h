@@ -14,25 +14,22 @@ constexpr int kMaxKvHeads = 256;
 // the current layer (the workspace is sized for nret = Hkv).
 struct Workspace {
   float* scores;                  // [slots][ld]             scaled indexer scores
-  float* chunk_max;               // [slots][n_score_chunks] per-CTA maxima of the scores
+  float* cta_max;                 // [slots][select_ctas]    per-CTA maxima of the scores
   unsigned long long* hist;       // [slots][256]            fixed-point (2^-40) bin masses
   float* s_max;                   // [slots]
   int* bstar;                     // [slots]
   unsigned long long* mass_total; // [slots]                 C_0 in fixed point
   int* sel_idx;                   // [slots][ld]             selected positions, ascending
-  uint32_t* chunk_bins;           // [slots][n_sel_chunks][256] tokens per bin and chunk
-  int* chunk_off;                 // [slots][n_sel_chunks+1] selected tokens before each chunk
+  uint32_t* cta_bins;             // [slots][select_ctas][256] tokens per bin, per scoring CTA
   int* sel_total;                 // [slots]                 |S|
   int* sel_n;                     // [slots]                 N the selection was made over
-  unsigned* ticket_hist;          // [slots]
+  unsigned* grid_bar;             // grid barrier of the selection kernel: generation, root, groups
   unsigned* ticket_attend;        // [B*Hkv]                 merge of a head's groups
   unsigned* ticket_group;         // [B*Hkv][n_merge_groups] merge of a group's pieces
   float* partials;                // [(attend_ctas + B*Hkv)][kPartFloats]  one per piece
   float* group_partials;          // [B*Hkv][n_merge_groups][kPartFloats]
   unsigned* status;               // [1] RTP_DEV_* bits
   int ld;                         // per-slot stride of scores / sel_idx: max_ctx rounded up to 64
-  int n_score_chunks;             // ceil(max_ctx / kScoreChunk)
-  int n_sel_chunks;               // ceil(max_ctx / kSelChunk)
   int n_merge_groups;             // ceil(attend_ctas / kMergeFanIn)
 };
 
@@ -47,15 +44,16 @@ struct LayerArgs {
   int* sel_count;                 // [B][Hkv] or nullptr
   int B, Hq, Hkv, G, max_ctx, window, sinks, nret;
   int dense;                      // every head attends over all N tokens
+  int heads;                      // attention launch: kHeadsAll, kHeadsLocal or kHeadsRetrieval
   float top_p, idx_scale, attn_scale_log2, bin_scale;
   short ret_kvh[kMaxKvHeads];     // KV head of retrieval index j (j < nret)
   short slot_of_kvh[kMaxKvHeads]; // retrieval index j of KV head kvh, or -1 for a local head
 };
 
+enum : int { kHeadsAll = 0, kHeadsLocal = 1, kHeadsRetrieval = 2 };
+
 // Kernel entry points (defined in select_kernels.cu / attend_kernel.cu).
-__global__ void score_kernel(const LayerArgs a, const Workspace w);
-__global__ void hist_kernel(const LayerArgs a, const Workspace w);
-__global__ void compact_kernel(const LayerArgs a, const Workspace w);
+__global__ void select_kernel(const LayerArgs a, const Workspace w);  // cooperative launch
 __global__ void attend_kernel(const LayerArgs a, const Workspace w);
 
 constexpr int kAttendWarps = 4;                          // warps per attention CTA
@@ -64,6 +62,10 @@ constexpr int kAttendCtasPerSm = 2;                      // resident attention C
 constexpr int kAttendThreads = kAttendWarps * 32;
 constexpr int kRowBytes = 128 * 2;                       // one K or V row
 constexpr int kMaxAttendHeads = 1024;                    // B * Hkv per layer
+constexpr int kMaxSelSlots = kMaxAttendHeads;            // retrieval slots per layer
+constexpr int kMaxSelectCtasPerSm = 2;                   // resident selection CTAs per SM
+constexpr int kScoreCap = 16384;                         // scores a selection CTA keeps on chip
+size_t select_smem_bytes(int slots);
 constexpr int kMergeFanIn = 16;                          // pieces merged per tree node
 // the attention grid is at most kMergeFanIn * 2 * kMergeFanIn CTAs (two merge levels)
 

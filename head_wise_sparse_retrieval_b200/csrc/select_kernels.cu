@@ -2,28 +2,34 @@
 //
 // Follows "Full Attention Strikes Back ..." (xllm-io paper review), section 三:
 //   核心公式 / 自适应稀疏注意力  s_h(m,n) = (W^Q q^pre)^T (W^K k^pre),  S_h(m) = Top-P(s_h, p)
-//   硬件感知解码内核            top-p without sorting, over a 256-bin histogram (O(1) per head)
+//   硬件感知解码内核            top-p without sorting, over a 256-bin histogram (O(1) per head),
+//                              scoring and selection in one launch
 // and the gist.science technical summary, Methodology 3 (mass accumulated until p is reached).
 //
-// Three launches per layer, each over (chunk, retrieval slot) with PDL between them:
-//   score_kernel   streams the N x 16 fp16 indexer keys once (two 16-byte loads per token,
-//                  a lane pair per token), writes the fp32 scaled scores (they stay in L2)
-//                  and one maximum per 1024-token chunk;
-//   hist_kernel    s_max = max of the chunk maxima; bins every score relative to s_max and
-//                  adds exp(s - s_max) to 256 shared bins in 2^-40 fixed point
-//                  (integer adds: the result does not depend on the order of arrival); the
-//                  last CTA of a slot (atomic ticket, no waiting) scans the bins from the top
-//                  with one warp and writes b*;
-//                  The same CTAs count tokens per bin and chunk, so once b* is known the last
-//                  CTA also writes how many tokens each chunk selects and their prefix;
-//   compact_kernel re-bins with the same function and writes the selected positions, in
-//                  ascending order, into one dense list (each chunk at its prefix offset).
-// Bins need the global s_max, so the scores make one round trip through L2 (4 B per token
-// against 32 B of indexer keys read from HBM).
+// One persistent cooperative launch per layer selects the tokens of every retrieval slot
+// (slot = b * nret + j for the j-th retrieval KV head). The indexer keys of all slots are laid
+// end to end and cut into one equal range per CTA; a CTA keeps the scores of its range in its
+// own shared memory (ranges longer than kScoreCap spill the rest to a global buffer). Three
+// phases, two grid barriers (bounded waits):
+//   1. scores: a lane pair reads a token's 32 bytes with two 16-byte loads (double-buffered),
+//      the scaled fp32 score is kept, and each CTA records the max of each slot it scores;
+//   2. histogram: s_max of a slot = max of its CTAs' maxima; every score is binned relative
+//      to s_max and exp(s - s_max) is added in 2^-40 fixed point to per-warp shared bins
+//      (32-bit words, exact integer sums whatever the order). The CTA adds its masses to the
+//      slot's global histogram (integer atomics) and stores its token count per bin;
+//   3. compaction: each CTA computes b* from the slot's histogram (one warp, suffix sums from
+//      the top bin), its offset from the bin counts (bins >= b*) of the CTAs before it, and
+//      writes its selected positions, ascending, into one dense list per slot.
+// Phases 2 and 3 bin the same fp32 scores with score_bin, so counts and flags agree exactly.
 #include "rtp_device.cuh"
 #include "rtp_kernels.h"
 
 namespace rtp {
+
+namespace {
+
+constexpr int kWarpsSel = kSelThreads / 32;
+constexpr int kRowUnroll = 16;  // independent 16-byte loads per thread in the offset sums
 
 __device__ __forceinline__ int clamp_seq_len(const LayerArgs& a, int b, unsigned* status,
                                              bool report) {
@@ -35,93 +41,34 @@ __device__ __forceinline__ int clamp_seq_len(const LayerArgs& a, int b, unsigned
   return n;
 }
 
-__device__ __forceinline__ float block_max_256(float v, float* red) {
+__device__ __forceinline__ float block_max(float v, float* red) {
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  __syncthreads();
   if (lane == 0) red[warp] = v;
   __syncthreads();
   float r = red[0];
 #pragma unroll
-  for (int i = 1; i < kSelThreads / 32; ++i) r = fmaxf(r, red[i]);
-  __syncthreads();
+  for (int i = 1; i < kWarpsSel; ++i) r = fmaxf(r, red[i]);
   return r;
 }
 
-// ---- 1. indexer scores -------------------------------------------------------------------
-
-__global__ void __launch_bounds__(kSelThreads) score_kernel(const LayerArgs a, const Workspace w) {
-  __shared__ float red[kSelThreads / 32];
-  pdl_wait();
-  const int slot = blockIdx.y;
-  const int b = slot / a.nret, kvh = a.ret_kvh[slot % a.nret];
-  const int N = clamp_seq_len(a, b, w.status, blockIdx.x == 0 && threadIdx.x == 0);
-
-  if (blockIdx.x == 0) {  // reset what the next two kernels accumulate into
-    w.hist[(size_t)slot * kBins + threadIdx.x] = 0ull;
-    if (threadIdx.x == 0) w.ticket_hist[slot] = 0u;
-  }
-  pdl_launch_dependents();
-
-  const int n0 = blockIdx.x * kScoreChunk;
-  if (n0 >= N) return;
-  const int n1 = min(n0 + kScoreChunk, N);
-
-  // a lane pair per token: the even lane holds dims 0..7, the odd lane dims 8..15
-  const int half = threadIdx.x & 1, pair = threadIdx.x >> 1;
-  const size_t head = (size_t)b * a.Hkv + kvh;
-  float q[8];
-  {
-    const uint4 qv = *reinterpret_cast<const uint4*>(a.q_idx + head * kIdxDim + half * 8);
-    const __half2* h2 = reinterpret_cast<const __half2*>(&qv);
+__device__ __forceinline__ int block_sum(int v, int* red) {
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      const float2 f = __half22float2(h2[i]);
-      q[2 * i] = f.x;
-      q[2 * i + 1] = f.y;
-    }
-  }
-  const uint4* keys = reinterpret_cast<const uint4*>(a.k_idx + head * (size_t)a.max_ctx * kIdxDim);
-  float* sc = w.scores + (size_t)slot * w.ld;
-
-  constexpr int kIter = kScoreChunk / (kSelThreads / 2);  // 8 tokens per lane pair
-  uint4 kv[kIter];
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  __syncthreads();
+  if (lane == 0) red[warp] = v;
+  __syncthreads();
+  int r = 0;
 #pragma unroll
-  for (int it = 0; it < kIter; ++it) {
-    const int n = n0 + it * (kSelThreads / 2) + pair;
-    kv[it] = (n < n1) ? __ldcs(keys + 2 * (size_t)n + half) : make_uint4(0, 0, 0, 0);
-  }
-  float mx = -INFINITY;
-#pragma unroll
-  for (int it = 0; it < kIter; ++it) {
-    const int n = n0 + it * (kSelThreads / 2) + pair;
-    const __half2* h2 = reinterpret_cast<const __half2*>(&kv[it]);
-    float p[8];
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      const float2 f = __half22float2(h2[i]);
-      p[2 * i] = __fmul_rn(q[2 * i], f.x);       // fp16 x fp16 products are exact in fp32
-      p[2 * i + 1] = __fmul_rn(q[2 * i + 1], f.y);
-    }
-    // pairwise sum: 8 products, then the partner lane's 8
-    const float s01 = __fadd_rn(p[0], p[1]), s23 = __fadd_rn(p[2], p[3]);
-    const float s45 = __fadd_rn(p[4], p[5]), s67 = __fadd_rn(p[6], p[7]);
-    const float part = __fadd_rn(__fadd_rn(s01, s23), __fadd_rn(s45, s67));
-    const float other = __shfl_xor_sync(0xffffffffu, part, 1);
-    const float s = __fmul_rn(__fadd_rn(part, other), a.idx_scale);
-    if (n < n1) {
-      if (half == 0) sc[n] = s;
-      mx = fmaxf(mx, s);
-    }
-  }
-  mx = block_max_256(mx, red);
-  if (threadIdx.x == 0) w.chunk_max[(size_t)slot * w.n_score_chunks + blockIdx.x] = mx;
+  for (int i = 0; i < kWarpsSel; ++i) r += red[i];
+  return r;
 }
 
-// ---- 2. mass histogram + threshold bin + chunk offsets ------------------------------------
-
-// Block-wide exclusive scan of one int per thread (256 threads); returns the block total.
-__device__ __forceinline__ int block_excl_scan_256(int v, int& excl, int* warp_tot) {
+// Block-wide exclusive scan of one int per thread; returns the block total.
+__device__ __forceinline__ int block_excl_scan(int v, int& excl, int* red) {
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   int x = v;
 #pragma unroll
@@ -129,215 +76,359 @@ __device__ __forceinline__ int block_excl_scan_256(int v, int& excl, int* warp_t
     const int y = __shfl_up_sync(0xffffffffu, x, o);
     if (lane >= o) x += y;
   }
-  if (lane == 31) warp_tot[warp] = x;
+  __syncthreads();
+  if (lane == 31) red[warp] = x;
   __syncthreads();
   int before = 0, all = 0;
 #pragma unroll
-  for (int k = 0; k < kSelThreads / 32; ++k) {
-    const int t = warp_tot[k];
+  for (int k = 0; k < kWarpsSel; ++k) {
+    const int t = red[k];
     before += (k < warp) ? t : 0;
     all += t;
   }
-  __syncthreads();
   excl = before + x - v;
   return all;
 }
 
-// Loads the kPerThread consecutive scores of this thread (positions n..n+kPerThread-1), with
-// -inf past n1.
-__device__ __forceinline__ void load_scores(const float* sc, int n, int n1, float (&v)[kPerThread]) {
-  if (n + kPerThread <= n1) {
-#pragma unroll
-    for (int k = 0; k < kPerThread; k += 4) {
-      const float4 f = __ldcg(reinterpret_cast<const float4*>(sc + n + k));
-      v[k] = f.x;
-      v[k + 1] = f.y;
-      v[k + 2] = f.z;
-      v[k + 3] = f.w;
-    }
-  } else {
-#pragma unroll
-    for (int k = 0; k < kPerThread; ++k) v[k] = (n + k < n1) ? __ldcg(sc + n + k) : -INFINITY;
-  }
-}
-
-__global__ void __launch_bounds__(kSelThreads) hist_kernel(const LayerArgs a, const Workspace w) {
-  // Per-warp histograms of the 2^-40 fixed-point masses, split into 32-bit low and high words
-  // (native shared-memory atomics; the carry of the low word is detected from the returned old
-  // value), and one token-count histogram. Integer sums: exact, independent of arrival order.
-  constexpr int kWarps = kSelThreads / 32;
-  __shared__ uint32_t wlo[kWarps][kBins];
-  __shared__ uint32_t whi[kWarps][kBins];
-  __shared__ uint32_t cnt[kBins];
-  __shared__ float red[kWarps];
-  __shared__ int warp_tot[kWarps];
-  __shared__ int is_last, bstar_s, carry_s;
-  for (int i = threadIdx.x; i < kWarps * kBins; i += kSelThreads) {
-    (&wlo[0][0])[i] = 0u;  // before the dependency wait: overlaps the previous kernel
-    (&whi[0][0])[i] = 0u;
-  }
-  cnt[threadIdx.x] = 0u;
-  pdl_wait();
-  pdl_launch_dependents();
-
-  const int slot = blockIdx.y;
-  const int b = slot / a.nret;
-  const int N = clamp_seq_len(a, b, w.status, false);
-  const int n0 = blockIdx.x * kSelChunk;
-  if (n0 >= N) return;
-  const int n1 = min(n0 + kSelChunk, N);
-  const int warp = threadIdx.x >> 5;
-
-  // s_max over the chunk maxima of the whole context (max is order-independent)
-  const int nsc = (N + kScoreChunk - 1) / kScoreChunk;
-  float m = -INFINITY;
-  for (int i = threadIdx.x; i < nsc; i += kSelThreads)
-    m = fmaxf(m, __ldcg(w.chunk_max + (size_t)slot * w.n_score_chunks + i));
-  const float s_max = block_max_256(m, red);  // also orders the zero fill before the adds
-
-  const float* sc = w.scores + (size_t)slot * w.ld;
-  float sv[kPerThread];
-  load_scores(sc, n0 + threadIdx.x * kPerThread, n1, sv);
-  uint32_t* lo_h = wlo[warp];
-  uint32_t* hi_h = whi[warp];
-#pragma unroll
-  for (int k = 0; k < kPerThread; ++k) {
-    const float s = sv[k];
-    if (s == -INFINITY) continue;
-    const int bin = score_bin(s, s_max, a.bin_scale);
-    const float wgt = expf(s - s_max);                       // in (0, 1]
-    const unsigned long long fx = __float2ull_rn(wgt * 1099511627776.0f);  // * 2^40, exact
-    const uint32_t lo = (uint32_t)fx;
-    uint32_t hi = (uint32_t)(fx >> 32);
-    if (lo) {
-      const uint32_t old = atomicAdd(lo_h + bin, lo);
-      hi += (old + lo < old) ? 1u : 0u;                      // carry out of the low word
-    }
-    if (hi) atomicAdd(hi_h + bin, hi);
-    atomicAdd(cnt + bin, 1u);
-  }
+// Grid-wide barrier of a cooperative launch (every CTA is resident). Arrivals go through one
+// counter per group of kBarGroup CTAs, then the group's last arrival through the root counter;
+// the root's last arrival bumps the generation word. The wait gives up after kWaitLimitNs, sets
+// kDevWaitTimeout and makes later barriers of the CTA return at once, so the kernel ends.
+// bar: [0] generation, [1] root counter, [2 ..] group counters.
+constexpr int kBarGroup = 16;
+__device__ void grid_barrier(unsigned* bar, unsigned* status, int* aborted) {
   __syncthreads();
-  {
-    unsigned long long v = 0ull;
-#pragma unroll
-    for (int k = 0; k < kWarps; ++k)
-      v += ((unsigned long long)whi[k][threadIdx.x] << 32) + wlo[k][threadIdx.x];
-    if (v) atomicAdd(w.hist + (size_t)slot * kBins + threadIdx.x, v);
-    w.chunk_bins[((size_t)slot * w.n_sel_chunks + blockIdx.x) * kBins + threadIdx.x] =
-        cnt[threadIdx.x];
-  }
-  __threadfence();
-  __syncthreads();
-  if (threadIdx.x == 0) {
-    const unsigned nhc = (unsigned)((N + kSelChunk - 1) / kSelChunk);
-    is_last = (atomicAdd(w.ticket_hist + slot, 1u) == nhc - 1u);
-    carry_s = 0;
-  }
-  __syncthreads();
-  if (!is_last) return;
-  __threadfence();
-
-  // ---- last CTA of this slot: b* by one warp (8 bins per lane, suffix sums from the top) ----
-  if (threadIdx.x < 32) {
-    const int lane = threadIdx.x;
-    unsigned long long v[8], lane_sum = 0ull;
-#pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      v[i] = __ldcg(w.hist + (size_t)slot * kBins + lane * 8 + i);
-      lane_sum += v[i];
-    }
-    unsigned long long incl = lane_sum;  // sum over lanes >= lane
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-      const unsigned long long y = __shfl_down_sync(0xffffffffu, incl, o);
-      if (lane + o < 32) incl += y;
-    }
-    const unsigned long long total = __shfl_sync(0xffffffffu, incl, 0);
-    const double target = (double)a.top_p * (double)total;
-    unsigned long long c = incl - lane_sum;  // mass of the bins above this lane's
-    int best = -1;
-#pragma unroll
-    for (int i = 7; i >= 0; --i) {
-      c += v[i];
-      if (best < 0 && (double)c >= target) best = lane * 8 + i;
-    }
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) best = max(best, __shfl_xor_sync(0xffffffffu, best, o));
-    if (lane == 0) {
-      bstar_s = best < 0 ? 0 : best;
-      w.mass_total[slot] = total;
-    }
-  }
-  __syncthreads();
-  const int bs = bstar_s;
-
-  // ---- selected tokens per chunk (bins >= b*) and their exclusive prefix ----
-  const int nch = (N + kSelChunk - 1) / kSelChunk;
-  int* off = w.chunk_off + (size_t)slot * (w.n_sel_chunks + 1);
-  for (int base = 0; base < nch; base += kSelThreads) {
-    const int cc = base + threadIdx.x;
-    int v = 0;
-    if (cc < nch) {
-      const uint32_t* row = w.chunk_bins + ((size_t)slot * w.n_sel_chunks + cc) * kBins;
-      int bb = bs;
-      for (; bb < kBins && (bb & 3); ++bb) v += (int)__ldcg(row + bb);
-      for (; bb < kBins; bb += 4) {
-        const uint4 q = __ldcg(reinterpret_cast<const uint4*>(row + bb));
-        v += (int)(q.x + q.y + q.z + q.w);
+  if (threadIdx.x == 0 && !*aborted) {
+    const unsigned gen = ld_acquire_gpu(bar);
+    __threadfence();
+    const unsigned grp = blockIdx.x / kBarGroup;
+    const unsigned ngrp = (gridDim.x + kBarGroup - 1) / kBarGroup;
+    const unsigned in_grp = min((unsigned)kBarGroup, gridDim.x - grp * kBarGroup);
+    bool released = false;
+    if (atomicAdd(bar + 2 + grp, 1u) == in_grp - 1u) {
+      atomicExch(bar + 2 + grp, 0u);
+      if (atomicAdd(bar + 1, 1u) == ngrp - 1u) {
+        atomicExch(bar + 1, 0u);
+        __threadfence();
+        atomicAdd(bar, 1u);
+        released = true;
       }
     }
-    int excl;
-    const int all = block_excl_scan_256(v, excl, warp_tot);
-    const int carry = carry_s;
-    if (cc < nch) off[cc] = carry + excl;
-    __syncthreads();
-    if (threadIdx.x == 0) carry_s = carry + all;
-    __syncthreads();
+    if (!released) {
+      const unsigned long long t0 = global_ns();
+      unsigned it = 0;
+      while (ld_acquire_gpu(bar) == gen) {
+        if ((++it & 255u) == 0 && global_ns() - t0 > kWaitLimitNs) {
+          atomicOr(status, kDevWaitTimeout);
+          *aborted = 1;
+          break;
+        }
+      }
+    }
+    __threadfence();
   }
-  if (threadIdx.x == 0) {
-    const int total = carry_s;
-    off[nch] = total;
-    w.bstar[slot] = bs;
-    w.s_max[slot] = s_max;
-    w.sel_total[slot] = total;
-    w.sel_n[slot] = N;
-    w.ticket_hist[slot] = 0u;
-  }
+  __syncthreads();
 }
 
-// ---- 3. compaction: the selected positions, ascending, into one dense list -----------------
+// Largest s < S with off[s] <= x (off ascending, off[0] = 0 <= x < off[S]).
+__device__ __forceinline__ int upper_slot(const long long* off, int S, long long x) {
+  int lo = 0, hi = S - 1;
+  while (lo < hi) {
+    const int mid = (lo + hi + 1) >> 1;
+    if (off[mid] <= x) lo = mid; else hi = mid - 1;
+  }
+  return lo;
+}
 
-__global__ void __launch_bounds__(kSelThreads) compact_kernel(const LayerArgs a,
-                                                              const Workspace w) {
-  __shared__ int warp_tot[kSelThreads / 32];
+// CTA whose range [floor(c T / P), floor((c+1) T / P)) holds position x (0 <= x < T, P <= T).
+__device__ __forceinline__ long long cta_of(long long x, long long T, long long P) {
+  return ((x + 1) * P + T - 1) / T - 1;
+}
+
+// The scores of this CTA's range: the first kScoreCap in shared memory, the rest (if any) in
+// the global buffer at their slot positions.
+struct Scores {
+  float* sm;        // shared, indexed by position in the CTA range
+  float* glob;      // global scores workspace
+  size_t ld;
+  long long t0;     // range start (concatenated coordinates)
+  const long long* soff;
+  __device__ float* at(int s, int n) const {
+    const long long i = soff[s] + n - t0;
+    return (i < kScoreCap) ? sm + i : glob + (size_t)s * ld + n;
+  }
+};
+
+}  // namespace
+
+size_t select_smem_bytes(int slots) {
+  return (size_t)kScoreCap * 4 + (size_t)(slots + 1) * 8;
+}
+
+__global__ void __launch_bounds__(kSelThreads, 2) select_kernel(const LayerArgs a, const Workspace w) {
+  extern __shared__ __align__(16) unsigned char dsm[];
+  __shared__ uint32_t wlo[kWarpsSel][kBins];   // per-warp fixed-point masses, low words
+  __shared__ uint32_t whi[kWarpsSel][kBins];   // high words
+  __shared__ uint32_t cnt[kBins];              // tokens per bin in the segment
+  __shared__ float redf[kWarpsSel];
+  __shared__ int redi[kWarpsSel];
+  __shared__ int aborted;
+  __shared__ int bstar_s;
+
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int S = a.B * a.nret;
+  float* s_scores = reinterpret_cast<float*>(dsm);
+  long long* soff = reinterpret_cast<long long*>(dsm + (size_t)kScoreCap * 4);
+  if (tid == 0) aborted = 0;
   pdl_wait();
   pdl_launch_dependents();
 
-  const int slot = blockIdx.y;
-  const int b = slot / a.nret;
-  const int N = clamp_seq_len(a, b, w.status, false);
-  const int n0 = blockIdx.x * kSelChunk;
-  if (n0 >= N) return;
-  const int n1 = min(n0 + kSelChunk, N);
-  const int bstar = __ldcg(w.bstar + slot);
-  const float s_max = __ldcg(w.s_max + slot);
-  const int base = __ldcg(w.chunk_off + (size_t)slot * (w.n_sel_chunks + 1) + blockIdx.x);
-  const float* sc = w.scores + (size_t)slot * w.ld;
-  int* out = w.sel_idx + (size_t)slot * w.ld;
+  // slot sizes and their prefix sums
+  for (int s = tid; s < S; s += kSelThreads)
+    soff[s + 1] = clamp_seq_len(a, s / a.nret, w.status, blockIdx.x == 0 && (s % a.nret) == 0);
+  __syncthreads();
+  if (warp == 0) {  // inclusive scan, 32 slots at a time
+    long long carry = 0;
+    for (int base = 0; base < S; base += 32) {
+      const int i = base + lane;
+      long long x = (i < S) ? soff[i + 1] : 0;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const long long y = __shfl_up_sync(0xffffffffu, x, o);
+        if (lane >= o) x += y;
+      }
+      if (i < S) soff[i + 1] = carry + x;
+      carry += __shfl_sync(0xffffffffu, x, 31);
+    }
+    if (lane == 0) soff[0] = 0;
+  }
+  if (blockIdx.x == 0)  // phase 2 accumulates into these
+    for (int i = tid; i < S * kBins; i += kSelThreads) w.hist[i] = 0ull;
+  __syncthreads();
 
-  const int n = n0 + threadIdx.x * kPerThread;  // this thread's kPerThread consecutive tokens
-  float sv[kPerThread];
-  load_scores(sc, n, n1, sv);
-  unsigned flags = 0u;
+  const long long T = soff[S];
+  const long long P = min((long long)gridDim.x, T);
+  const bool active = (long long)blockIdx.x < P;
+  const long long t0 = active ? (long long)blockIdx.x * T / P : 0;
+  const long long t1 = active ? ((long long)blockIdx.x + 1) * T / P : 0;
+  const Scores sc{s_scores, w.scores, (size_t)w.ld, t0, soff};
+
+  // ---- phase 1: indexer scores of this CTA's range -----------------------------------------
+  if (active) {
+    int s = upper_slot(soff, S, t0);
+    const int half = tid & 1, pair = tid >> 1;
+    for (long long t = t0; t < t1; ++s) {
+      const int n0 = (int)(t - soff[s]);
+      const int n1 = (int)(min(t1, soff[s + 1]) - soff[s]);
+      t = soff[s] + n1;
+      const int b = s / a.nret, kvh = a.ret_kvh[s % a.nret];
+      const size_t head = (size_t)b * a.Hkv + kvh;
+      float q[8];
+      {
+        const uint4 qv = *reinterpret_cast<const uint4*>(a.q_idx + head * kIdxDim + half * 8);
+        const __half2* h2 = reinterpret_cast<const __half2*>(&qv);
 #pragma unroll
-  for (int k = 0; k < kPerThread; ++k)
-    if (sv[k] != -INFINITY && score_bin(sv[k], s_max, a.bin_scale) >= bstar) flags |= 1u << k;
-  int excl;
-  block_excl_scan_256(__popc(flags), excl, warp_tot);
-  int at = base + excl;
+        for (int i = 0; i < 4; ++i) {
+          const float2 f = __half22float2(h2[i]);
+          q[2 * i] = f.x;
+          q[2 * i + 1] = f.y;
+        }
+      }
+      const uint4* keys =
+          reinterpret_cast<const uint4*>(a.k_idx + head * (size_t)a.max_ctx * kIdxDim);
+      constexpr int kPairs = kSelThreads / 2, kUnroll = 8;
+      float mx = -INFINITY;
+      uint4 kv[kUnroll], nx[kUnroll];
+      auto load_batch = [&](uint4 (&dst)[kUnroll], int base) {
 #pragma unroll
-  for (int k = 0; k < kPerThread; ++k)
-    if (flags & (1u << k)) out[at++] = n + k;
+        for (int u = 0; u < kUnroll; ++u) {
+          const int n = base + u * kPairs + pair;
+          dst[u] = (n < n1) ? __ldcs(keys + 2 * (size_t)n + half) : make_uint4(0, 0, 0, 0);
+        }
+      };
+      load_batch(kv, n0);
+      for (int base = n0; base < n1; base += kPairs * kUnroll) {
+        if (base + kPairs * kUnroll < n1) load_batch(nx, base + kPairs * kUnroll);  // prefetch
+#pragma unroll
+        for (int u = 0; u < kUnroll; ++u) {
+          const int n = base + u * kPairs + pair;
+          const __half2* h2 = reinterpret_cast<const __half2*>(&kv[u]);
+          float p[8];
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            const float2 f = __half22float2(h2[i]);
+            p[2 * i] = __fmul_rn(q[2 * i], f.x);      // fp16 x fp16 products are exact in fp32
+            p[2 * i + 1] = __fmul_rn(q[2 * i + 1], f.y);
+          }
+          // pairwise sum: 8 products, then the partner lane's 8
+          const float s01 = __fadd_rn(p[0], p[1]), s23 = __fadd_rn(p[2], p[3]);
+          const float s45 = __fadd_rn(p[4], p[5]), s67 = __fadd_rn(p[6], p[7]);
+          const float part = __fadd_rn(__fadd_rn(s01, s23), __fadd_rn(s45, s67));
+          const float other = __shfl_xor_sync(0xffffffffu, part, 1);
+          const float sv = __fmul_rn(__fadd_rn(part, other), a.idx_scale);
+          if (n < n1) {
+            if (half == 0) *sc.at(s, n) = sv;
+            mx = fmaxf(mx, sv);
+          }
+        }
+#pragma unroll
+        for (int u = 0; u < kUnroll; ++u) kv[u] = nx[u];
+      }
+      mx = block_max(mx, redf);
+      if (tid == 0) w.cta_max[(size_t)s * gridDim.x + blockIdx.x] = mx;
+    }
+  }
+  grid_barrier(w.grid_bar, w.status, &aborted);
+
+  // ---- phase 2: mass histogram and token counts of this CTA's segments ---------------------
+  if (active) {
+    int s = upper_slot(soff, S, t0);
+    for (long long t = t0; t < t1; ++s) {
+      const int n0 = (int)(t - soff[s]);
+      const int n1 = (int)(min(t1, soff[s + 1]) - soff[s]);
+      t = soff[s] + n1;
+      const long long c0 = cta_of(soff[s], T, P), c1 = cta_of(soff[s + 1] - 1, T, P);
+      float m = -INFINITY;  // s_max of the slot: max over the CTAs that scored it
+      for (long long c = c0 + tid; c <= c1; c += kSelThreads)
+        m = fmaxf(m, __ldcg(w.cta_max + (size_t)s * gridDim.x + c));
+      for (int i = tid; i < kWarpsSel * kBins; i += kSelThreads) {
+        (&wlo[0][0])[i] = 0u;
+        (&whi[0][0])[i] = 0u;
+      }
+      cnt[tid] = 0u;
+      const float s_max = block_max(m, redf);  // its barriers also order the zero fill
+      for (int n = n0 + tid; n < n1; n += kSelThreads) {
+        const float v = *sc.at(s, n);
+        const int bin = score_bin(v, s_max, a.bin_scale);
+        const float wgt = expf(v - s_max);                          // in (0, 1]
+        const unsigned long long fx = __float2ull_rn(wgt * 1099511627776.0f);  // * 2^40, exact
+        const uint32_t lo = (uint32_t)fx;
+        uint32_t hi = (uint32_t)(fx >> 32);
+        if (lo) {
+          const uint32_t old = atomicAdd(&wlo[warp][bin], lo);
+          hi += (old + lo < old) ? 1u : 0u;                          // carry out of the low word
+        }
+        if (hi) atomicAdd(&whi[warp][bin], hi);
+        atomicAdd(&cnt[bin], 1u);
+      }
+      __syncthreads();
+      unsigned long long v = 0ull;
+#pragma unroll
+      for (int k = 0; k < kWarpsSel; ++k)
+        v += ((unsigned long long)whi[k][tid] << 32) + wlo[k][tid];
+      if (v) atomicAdd(w.hist + (size_t)s * kBins + tid, v);
+      w.cta_bins[((size_t)s * gridDim.x + blockIdx.x) * kBins + tid] = cnt[tid];
+      if (blockIdx.x == c0 && tid == 0) w.s_max[s] = s_max;
+      __syncthreads();
+    }
+  }
+  grid_barrier(w.grid_bar, w.status, &aborted);
+
+  // ---- phase 3: b*, offsets and the dense selected list -----------------------------------
+  if (active) {
+    int s = upper_slot(soff, S, t0);
+    for (long long t = t0; t < t1; ++s) {
+      const int n0 = (int)(t - soff[s]);
+      const int n1 = (int)(min(t1, soff[s + 1]) - soff[s]);
+      t = soff[s] + n1;
+      const int c0 = (int)cta_of(soff[s], T, P), c1 = (int)cta_of(soff[s + 1] - 1, T, P);
+      const bool first = (int)blockIdx.x == c0;
+      if (warp == 0) {  // b*: one warp, 8 bins per lane, suffix sums from the top bin down
+        unsigned long long hv[8], lane_sum = 0ull;
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          hv[i] = __ldcg(w.hist + (size_t)s * kBins + lane * 8 + i);
+          lane_sum += hv[i];
+        }
+        unsigned long long incl = lane_sum;  // sum over lanes >= lane
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+          const unsigned long long y = __shfl_down_sync(0xffffffffu, incl, o);
+          if (lane + o < 32) incl += y;
+        }
+        const unsigned long long total = __shfl_sync(0xffffffffu, incl, 0);
+        const double target = (double)a.top_p * (double)total;
+        unsigned long long c = incl - lane_sum;  // mass of the bins above this lane's
+        int best = -1;
+#pragma unroll
+        for (int i = 7; i >= 0; --i) {
+          c += hv[i];
+          if (best < 0 && (double)c >= target) best = lane * 8 + i;
+        }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) best = max(best, __shfl_xor_sync(0xffffffffu, best, o));
+        if (lane == 0) {
+          bstar_s = best < 0 ? 0 : best;
+          if (first) w.mass_total[s] = total;
+        }
+      }
+      __syncthreads();
+      const int bs = bstar_s;
+      // selected tokens of the slot's CTAs before this one (first CTA: of all, for |S|); the
+      // (CTA, 4-bin group) pairs are spread over the threads so their 16-byte loads overlap
+      const int r0 = c0, r1 = first ? c1 + 1 : (int)blockIdx.x;
+      const int b4 = bs & ~3, ngrp = (kBins - b4) >> 2;
+      const uint32_t* rows_base = w.cta_bins + (size_t)s * gridDim.x * kBins + b4;
+      const int E = (r1 - r0) * ngrp;
+      int mine = 0;
+      for (int e0 = 0; e0 < E; e0 += kSelThreads * kRowUnroll) {
+        uint4 q4[kRowUnroll];
+#pragma unroll
+        for (int k = 0; k < kRowUnroll; ++k) {
+          const int e = e0 + k * kSelThreads + tid;
+          q4[k] = (e < E) ? __ldcg(reinterpret_cast<const uint4*>(
+                                rows_base + (size_t)(r0 + e / ngrp) * kBins + (e % ngrp) * 4))
+                          : make_uint4(0, 0, 0, 0);
+        }
+#pragma unroll
+        for (int k = 0; k < kRowUnroll; ++k) {
+          const int e = e0 + k * kSelThreads + tid;
+          if ((e % ngrp) == 0) {  // first group of a row: drop the bins below b*
+            const int lo = bs - b4;
+            q4[k].x = (lo > 0) ? 0u : q4[k].x;
+            q4[k].y = (lo > 1) ? 0u : q4[k].y;
+            q4[k].z = (lo > 2) ? 0u : q4[k].z;
+          }
+          mine += (int)(q4[k].x + q4[k].y + q4[k].z + q4[k].w);
+        }
+      }
+      const int sum_rows = block_sum(mine, redi);
+      int base = first ? 0 : sum_rows;
+      if (first && tid == 0) {
+        w.bstar[s] = bs;
+        w.sel_total[s] = sum_rows;
+        w.sel_n[s] = (int)(soff[s + 1] - soff[s]);
+      }
+      const float s_max = __ldcg(w.s_max + s);
+      int* out = w.sel_idx + (size_t)s * w.ld;
+      // ordered compaction: warp w takes 32 x kPerThread consecutive tokens of each round, one
+      // ballot per 32; the warps' counts are scanned, then each warp writes its tokens in order
+      constexpr int kWarpSpan = 32 * kPerThread;
+      for (int rb = n0; rb < n1; rb += kWarpsSel * kWarpSpan) {
+        const int wb = rb + warp * kWarpSpan;
+        unsigned bal[kPerThread];
+        int wcnt = 0;
+#pragma unroll
+        for (int k = 0; k < kPerThread; ++k) {
+          const int n = wb + 32 * k + lane;
+          const bool f = n < n1 && score_bin(*sc.at(s, n), s_max, a.bin_scale) >= bs;
+          bal[k] = __ballot_sync(0xffffffffu, f);
+          wcnt += __popc(bal[k]);
+        }
+        int wexcl;
+        const int all = block_excl_scan(lane == 0 ? wcnt : 0, wexcl, redi);
+        int at = base + __shfl_sync(0xffffffffu, wexcl, 0);
+        const unsigned lt = (1u << lane) - 1u;
+#pragma unroll
+        for (int k = 0; k < kPerThread; ++k) {
+          if (bal[k] & (1u << lane)) out[at + __popc(bal[k] & lt)] = wb + 32 * k + lane;
+          at += __popc(bal[k]);
+        }
+        base += all;
+      }
+      __syncthreads();
+    }
+  }
 }
 
 }  // namespace rtp

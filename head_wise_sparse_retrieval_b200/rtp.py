@@ -25,7 +25,7 @@ EXPORTS = ("rtp_config_default", "rtp_workspace_bytes", "rtp_create", "rtp_destr
            "rtp_decode_step", "rtp_dense_decode", "rtp_decode_step_host", "rtp_get_selection",
            "rtp_get_threshold", "rtp_get_device_status", "rtp_status_string", "rtp_last_error",
            "rtp_profile_enable", "rtp_profile_read")
-KERNEL_CLASSES = ("score", "hist", "compact", "attend")
+KERNEL_CLASSES = ("select", "attend", "reserved2", "reserved3")
 
 
 class RtpError(RuntimeError):

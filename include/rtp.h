@@ -120,7 +120,8 @@ typedef struct {
                                 |T| for local heads; NULL to skip                                */
 } rtp_layer_io;
 
-/* Enqueues one layer of the decode step on `stream`. Asynchronous: no host synchronisation,
+/* Enqueues one layer of the decode step on `stream` (two kernels when the layer has retrieval
+ * heads: the selection, then the attention of every head). Asynchronous: no host synchronisation,
  * no allocation, capturable in a CUDA graph (the mask is read on the host at call time and the
  * launch shapes depend only on cfg and the mask). Errors (nothing enqueued): RTP_ERR_INVALID_ARG
  * for a NULL handle / io / required pointer, a misaligned device pointer, top_p outside (0, 1]
@@ -160,9 +161,9 @@ RTP_API rtp_status rtp_get_threshold(rtp_handle *h, int b, int kvh, int *bstar, 
 /* Kernel profiling. While enabled, every kernel that rtp_decode_step / rtp_dense_decode
  * launches on this handle is bracketed by two CUDA events recorded on the launch stream (the
  * events are created here, so the decode calls still allocate nothing). Do not enable it while
- * capturing a CUDA graph. Kernel classes: 0 indexer score, 1 histogram + threshold,
- * 2 compaction, 3 attention. The event pool holds 1024 launches; rtp_profile_read empties it.
- * Errors: RTP_ERR_CUDA if the events cannot be created. */
+ * capturing a CUDA graph. Kernel classes: 0 selection (indexer score, histogram top-p,
+ * compaction), 1 attention; 2 and 3 are reserved (always 0). The event pool holds 1024
+ * launches; rtp_profile_read empties it. Errors: RTP_ERR_CUDA if the events cannot be created. */
 RTP_API rtp_status rtp_profile_enable(rtp_handle *h, int enable);
 
 /* Synchronises the recorded launches, adds their durations (ms) and counts per kernel class

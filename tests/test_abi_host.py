@@ -41,7 +41,9 @@ def test_config_default_matches_pages(rtp_lib):
 def test_workspace_is_linear_in_context(rtp_lib):
     a = rtp_lib.workspace_bytes(rtp_lib.default_config(1, 1, 32, 4, 1 << 18))
     b = rtp_lib.workspace_bytes(rtp_lib.default_config(1, 1, 32, 4, 1 << 20))
-    assert a > 0 and 3.5 < b / a < 4.2
+    c = rtp_lib.workspace_bytes(rtp_lib.default_config(1, 1, 32, 4, 1 << 21))
+    # linear in max_ctx: b - a covers 3 * 2^18 more tokens, c - b covers 4 * 2^18
+    assert 0 < a < b < c and abs(3 * (c - b) - 4 * (b - a)) < 0.05 * (c - b)
     assert rtp_lib.workspace_bytes(rtp_lib.default_config(1, 1, 32, 4, 0)) == 0
 
 
