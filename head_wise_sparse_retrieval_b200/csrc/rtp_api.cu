@@ -247,6 +247,11 @@ struct DeviceGuard {
 
 }  // namespace
 
+namespace rtp {
+// Records the reason returned by rtp_last_error on this thread (used by noalloc.cu).
+void set_last_error(const char* msg) { snprintf(g_err, sizeof g_err, "%s", msg); }
+}  // namespace rtp
+
 extern "C" {
 
 void rtp_config_default(rtp_config* c, int num_layers, int batch, int num_q_heads,

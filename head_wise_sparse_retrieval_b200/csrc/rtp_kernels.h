@@ -70,5 +70,6 @@ constexpr int kMergeFanIn = 16;                          // pieces merged per tr
 // the attention grid is at most kMergeFanIn * 2 * kMergeFanIn CTAs (two merge levels)
 
 size_t attend_smem_bytes(int nheads, int batch);
+void set_last_error(const char* msg);  // the reason rtp_last_error reports on this thread
 
 }  // namespace rtp

@@ -24,7 +24,8 @@ DEV_BAD_SEQLEN, DEV_WAIT_TIMEOUT, DEV_BAD_INDEX = 0x1, 0x2, 0x4
 EXPORTS = ("rtp_config_default", "rtp_workspace_bytes", "rtp_create", "rtp_destroy",
            "rtp_decode_step", "rtp_dense_decode", "rtp_decode_step_host", "rtp_get_selection",
            "rtp_get_threshold", "rtp_get_device_status", "rtp_status_string", "rtp_last_error",
-           "rtp_profile_enable", "rtp_profile_read")
+           "rtp_profile_enable", "rtp_profile_read", "rtp_window_attention_noalloc")
+NOALLOC_MAX_HEADS = 64
 KERNEL_CLASSES = ("select", "attend", "reserved2", "reserved3")
 
 
@@ -41,6 +42,14 @@ class Config(ctypes.Structure):
         ("max_ctx", ctypes.c_int), ("window", ctypes.c_int), ("sinks", ctypes.c_int),
         ("num_bins", ctypes.c_int), ("idx_range", ctypes.c_float),
         ("idx_scale", ctypes.c_float), ("attn_scale", ctypes.c_float),
+    ]
+
+
+class NoAllocParams(ctypes.Structure):
+    _fields_ = [
+        ("batch", ctypes.c_int), ("num_q_heads", ctypes.c_int), ("num_kv_heads", ctypes.c_int),
+        ("max_ctx", ctypes.c_int), ("window", ctypes.c_int), ("sinks", ctypes.c_int),
+        ("attn_scale", ctypes.c_float), ("dense", ctypes.c_int),
     ]
 
 
@@ -84,6 +93,9 @@ def load(path: str = LIB_PATH):
     L.rtp_profile_enable.argtypes = [vp, i]
     L.rtp_profile_read.argtypes = [vp, ctypes.POINTER(ctypes.c_double),
                                    ctypes.POINTER(ctypes.c_int64)]
+    L.rtp_window_attention_noalloc.argtypes = [ctypes.POINTER(NoAllocParams), vp, vp, vp, vp,
+                                               vp, vp]
+    L.rtp_window_attention_noalloc.restype = ctypes.c_int
     L.rtp_status_string.argtypes = [i]
     L.rtp_status_string.restype = ctypes.c_char_p
     L.rtp_last_error.argtypes = []
@@ -234,6 +246,22 @@ class Handle:
         if st not in (RTP_OK, RTP_ERR_DEVICE_STATUS):
             _check(st, "rtp_get_device_status")
         return int(code.value)
+
+
+def window_attention_noalloc(q, k_cache, v_cache, seq_lens, out, *, window: int = 8192,
+                             sinks: int = 4, attn_scale: float | None = None, dense: bool = False,
+                             stream=None):
+    """rtp_window_attention_noalloc: window + sink (or dense) attention for every KV head,
+    without a handle and without allocating: for callers that cannot call cudaMalloc. Shapes
+    are read from the tensors: q [B, Hq, 128], caches [B, Hkv, max_ctx, 128]."""
+    B, Hq, D = q.shape
+    _, Hkv, Nmax, _ = k_cache.shape
+    p = NoAllocParams(B, Hq, Hkv, Nmax, window, sinks,
+                      float(attn_scale if attn_scale is not None else D ** -0.5), int(dense))
+    _check(load().rtp_window_attention_noalloc(ctypes.byref(p), _ptr(q), _ptr(k_cache),
+                                               _ptr(v_cache), _ptr(seq_lens), _ptr(out),
+                                               _stream_ptr(stream)),
+           "rtp_window_attention_noalloc")
 
 
 def config_for(plan, **overrides) -> Config:

@@ -174,6 +174,44 @@ RTP_API rtp_status rtp_profile_read(rtp_handle *h, double *ms, int64_t *launches
  * Returns RTP_ERR_DEVICE_STATUS when a bit was set, RTP_OK otherwise. */
 RTP_API rtp_status rtp_get_device_status(rtp_handle *h, uint32_t *code);
 
+/* ---- Attention without any allocation --------------------------------------------------
+ * The pages describe no such call; it exists for callers that cannot allocate device memory:
+ * engines that plan every byte up front and hand out memory only from their own pool, and
+ * latency-critical paths where cudaMalloc (which may synchronise the device) must not run.
+ * rtp_create allocates a workspace; this entry point needs no handle: its only scratch (the
+ * split-K partials and merge tickets of the attention kernel) is a file-scope device array of
+ * RTP_NOALLOC_SCRATCH_BYTES that every GPU loading the library holds until the process exits.
+ *
+ * It computes, for every (b, KV head), the attention over the window + sink set of a local
+ * head (dense == 0) or over all N_b tokens (dense != 0), exactly as rtp_decode_step does for a
+ * local head and rtp_dense_decode for any head. Layouts as in rtp_layer_io: q bf16 [B][Hq][128],
+ * k_cache / v_cache bf16 [B][Hkv][max_ctx][128], seq_lens int32 [B] (device), out fp32
+ * [B][Hq][128]; device pointers, 16-byte aligned (seq_lens 4-byte aligned).
+ *
+ * Limits: batch * num_kv_heads <= RTP_NOALLOC_MAX_HEADS, G = Hq / Hkv in 1..8, max_ctx in
+ * [1, 2^28], window >= 1, sinks >= 0; larger sizes return RTP_ERR_UNSUPPORTED with a message.
+ * It calls no cudaMalloc / cudaFree and no allocating library routine. The first call on a
+ * device looks up the array's device address (cudaGetSymbolAddress) with that device current;
+ * make that first call before any stream capture. Every call shares the one array, which keeps
+ * the last call's contents; the call clears the tickets it needs (an async memset on `stream`).
+ * Calls that overlap on the GPU (different streams, or the same array used from two threads'
+ * streams at once) race on the array. Device-side problems (a seq_lens entry outside
+ * [1, max_ctx], which is clamped) are not reported by this call. */
+#define RTP_NOALLOC_MAX_HEADS 64
+#define RTP_NOALLOC_MAX_CTAS 296
+#define RTP_NOALLOC_SCRATCH_BYTES 8388608
+
+typedef struct {
+    int batch, num_q_heads, num_kv_heads, max_ctx, window, sinks;  /* head_dim is 128 */
+    float attn_scale;                                                /* e.g. 1/sqrt(128)  */
+    int dense;                                                       /* 0: window + sinks */
+} rtp_noalloc_params;
+
+RTP_API rtp_status rtp_window_attention_noalloc(const rtp_noalloc_params *p, const void *q,
+                                                const void *k_cache, const void *v_cache,
+                                                const int32_t *seq_lens, float *out,
+                                                void *stream);
+
 /* Static string for a status code. */
 RTP_API const char *rtp_status_string(rtp_status s);
 
