@@ -32,6 +32,12 @@ sys.path.insert(0, ROOT)
 
 METRIC = "decode steps/s and effective HBM GB/s (% of roofline) at 128K–1M ctx"
 ROW_BYTES = 2 * 128 * 2      # one token's K and V rows (bf16, head_dim 128)
+# DRAM traffic of attend_kernel from one ncu capture (profiles/attend_kernel_ctx_1m_layer.md):
+# ctx_1m layer 2, 448.91 MB read + 3.98 MB written for 869 997 tokens x 512 B of algorithmic
+# bytes. It is scaled to a bench launch by that launch's algorithmic bytes, and reported only
+# while the kernel source is the one that was captured.
+ATTEND_NCU = {"source_sha256_16": "889a4df29f9b7326", "traffic_bytes": 448.909056e6 + 3.97952e6,
+              "algorithmic_bytes": 869997 * 512}
 IDX_BYTES = 16 * 2           # one token's indexer key (fp16, 16 dims)
 
 
@@ -225,6 +231,9 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-dense", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--single-layer", type=int, default=None,
+                    help="profiling case: only this layer of the workload, decoded --reps times")
+    ap.add_argument("--reps", type=int, default=3)
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
 
@@ -253,6 +262,23 @@ def main():
 
     rtp.load()
     dev = torch.device("cuda", local if world > 1 else 0)
+    if args.single_layer is not None:  # small case for ncu captures (one layer, a few calls)
+        l = args.single_layer
+        li = W.make_layer(plan, l, dev)
+        h = rtp.Handle(rtp.config_for(plan), dev.index)
+        out = torch.empty((plan.batch, plan.num_q_heads, 128), dtype=torch.float32, device=dev)
+        cnt = torch.empty((plan.batch, plan.num_kv_heads), dtype=torch.int32, device=dev)
+        for _ in range(args.reps):
+            h.decode_step(l, rtp.layer_from(li), plan.retrieval[l], plan.top_p, out, cnt)
+        torch.cuda.synchronize()
+        status = h.device_status()
+        h.close()
+        print(json.dumps({"single_layer": l, "workload": plan.name, "reps": args.reps,
+                          "retrieval": plan.retrieval[l].tolist(),
+                          "token_sets": cnt.cpu().tolist(), "device_status": status}))
+        if status:
+            raise SystemExit(1)
+        return
     torch.cuda.set_device(dev)
     L, B, Hq, Hkv = plan.num_layers, plan.batch, plan.num_q_heads, plan.num_kv_heads
 
@@ -336,6 +362,11 @@ def main():
     att_bytes_per_launch = attend_bytes / L
     hbm, peak_kind = _peaks()
     att_gbs = att_bytes_per_launch / (att_ms * 1e-3) / 1e9
+    traffic = None
+    import hashlib
+    src = os.path.join(ROOT, "head_wise_sparse_retrieval_b200", "csrc", "attend_kernel.cu")
+    if hashlib.sha256(open(src, "rb").read()).hexdigest()[:16] == ATTEND_NCU["source_sha256_16"]:
+        traffic = att_bytes_per_launch * ATTEND_NCU["traffic_bytes"] / ATTEND_NCU["algorithmic_bytes"]
 
     # dense decode on the same caches (the speedup denominator)
     dense = None
@@ -431,7 +462,7 @@ def main():
         "bytes_breakdown": {"indexer": idx_bytes, "attend_kv": attend_bytes},
         "roofline": {"bound": "hbm", "kernel": "attend_kernel", "achieved": att_gbs,
                      "peak": hbm, "peak_kind": peak_kind, "unit": "GB/s",
-                     "frac": att_gbs / hbm, "traffic": None,
+                     "frac": att_gbs / hbm, "traffic": traffic,
                      "per_launch_ms": att_ms, "algorithmic_bytes_per_launch": att_bytes_per_launch},
         "kernels": kern,
         "selection": {"retrieval_heads": len(n_sel),
