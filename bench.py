@@ -309,7 +309,7 @@ def main():
         raise SystemExit(f"device status 0x{status:x} after the eager step")
     sel = [c.cpu().numpy() for c in cnts]
     total_bytes, attend_bytes, idx_bytes = step_bytes(plan, sel)
-    launches_per_step = sum(2 if plan.retrieval[l].any() else 1 for l in range(L))
+    launches_per_step = sum(3 if plan.retrieval[l].any() else 2 for l in range(L))  # [select,] attend, merge
 
     # capture the whole step as one CUDA graph
     g = torch.cuda.CUDAGraph()

@@ -18,10 +18,9 @@
 //     heads of the GQA group as N = 8, so every fetched row serves the whole group:
 //     S^T = K Q^T, online softmax in the log2 domain, P rounded to bf16 and transposed in
 //     registers (movmatrix), O^T += V^T P^T.
-// At the end of a head's piece the warps merge (m, l, O) through shared memory. A head split
-// over several CTAs writes one partial per CTA; a two-level tree of atomic tickets (fan-in 16,
-// nothing waits) lets the last CTA of each group and then of the head merge the partials in a
-// fixed order (log-sum-exp) and write the output.
+// At the end of a head's piece the warps merge (m, l, O) through shared memory. A head held by
+// one CTA is written out there; a head split over several CTAs leaves one partial per CTA, and
+// merge_kernel (the next launch on the stream) combines them by log-sum-exp in a fixed order.
 #include "rtp_device.cuh"
 #include "rtp_kernels.h"
 
@@ -35,8 +34,8 @@ constexpr int kDepth = kAttendDepth;
 constexpr int kWarpStage = 2 * kTile * kRowBytes;          // 16 K rows then 16 V rows
 constexpr int kOPitch = kHeadDim + 4;                      // padded row of the merge buffer
 constexpr int kCombFloats = kMaxGroup * kOPitch + kWarps * kMaxGroup * 2;
-constexpr int kMaxMerge = 2 * kMergeFanIn;                 // sources of one merge
-constexpr int kMergeBatch = 4;                             // sources loaded per round trip
+constexpr int kMergeRows = kMergeThreads / 8;              // pieces a merge pass loads at once
+constexpr int kMergeRegs = 8;                              // passes kept in registers
 
 // Shared memory: per-warp stages, the warp-merge buffer, then the head tables sized by the
 // layer (B * Hkv + 1 offsets, B lengths).
@@ -182,73 +181,6 @@ __device__ __forceinline__ void issue_tile(uint32_t stage, const HeadRef& h, int
   }
 }
 
-// Log-sum-exp merge of n partials (o[8][128], m[8], l[8]), n <= kMaxMerge, by the 128 threads
-// of the CTA. (m, l) of every source go through shared memory in one round trip; then thread
-// tid owns query head jq = tid / 16 and dimensions 8 (tid % 16) .. +7 and issues the 16-byte
-// loads of kMergeBatch sources at a time. final: out[jq][d] = O / L; otherwise dst receives a partial.
-__device__ void merge_partials(int n, int G, bool final, float* dst, const float* const* src,
-                               float (*mM)[kMaxGroup], float (*mF)[kMaxGroup], float* mL,
-                               int tid) {
-  __syncthreads();  // src[] written
-  for (int e = tid; e < n * 2 * kMaxGroup; e += kAttendThreads) {
-    const int i = e / (2 * kMaxGroup), r = e % (2 * kMaxGroup);
-    const float v = __ldcg(src[i] + kPartO + r);  // m[0..7] then l[0..7]
-    if (r < kMaxGroup) mM[i][r] = v; else mF[i][r - kMaxGroup] = v;
-  }
-  __syncthreads();
-  if (tid < G) {
-    float M = -INFINITY;
-    for (int i = 0; i < n; ++i) M = fmaxf(M, mM[i][tid]);
-    float L = 0.f;
-    for (int i = 0; i < n; ++i) {
-      const float f = exp2f(mM[i][tid] - M);
-      L += mF[i][tid] * f;
-      mF[i][tid] = f;  // the l slot now holds the scale factor of source i
-    }
-    mL[tid] = L;
-    mM[0][tid] = M;    // source 0's m is no longer needed
-  }
-  __syncthreads();
-  const int jq = tid >> 4, d0 = (tid & 15) * 8;
-  if (jq < G) {
-    float4 o0 = make_float4(0.f, 0.f, 0.f, 0.f), o1 = o0;
-    for (int i0 = 0; i0 < n; i0 += kMergeBatch) {
-      float4 v0[kMergeBatch], v1[kMergeBatch];
-#pragma unroll
-      for (int i = 0; i < kMergeBatch; ++i) {
-        if (i0 + i < n) {
-          const float4* p = reinterpret_cast<const float4*>(src[i0 + i] + jq * kHeadDim + d0);
-          v0[i] = __ldcg(p);
-          v1[i] = __ldcg(p + 1);
-        }
-      }
-#pragma unroll
-      for (int i = 0; i < kMergeBatch; ++i) {
-        if (i0 + i < n) {
-          const float f = mF[i0 + i][jq];
-          o0.x += v0[i].x * f; o0.y += v0[i].y * f; o0.z += v0[i].z * f; o0.w += v0[i].w * f;
-          o1.x += v1[i].x * f; o1.y += v1[i].y * f; o1.z += v1[i].z * f; o1.w += v1[i].w * f;
-        }
-      }
-    }
-    if (final) {
-      const float inv = 1.f / mL[jq];
-      float4* q = reinterpret_cast<float4*>(dst + (size_t)jq * kHeadDim + d0);
-      q[0] = make_float4(o0.x * inv, o0.y * inv, o0.z * inv, o0.w * inv);
-      q[1] = make_float4(o1.x * inv, o1.y * inv, o1.z * inv, o1.w * inv);
-    } else {
-      float4* q = reinterpret_cast<float4*>(dst + jq * kHeadDim + d0);
-      q[0] = o0;
-      q[1] = o1;
-      if ((tid & 15) == 0) {
-        dst[kPartO + jq] = mM[0][jq];
-        dst[kPartO + kMaxGroup + jq] = mL[jq];
-      }
-    }
-  }
-  __syncthreads();  // scratch reusable
-}
-
 }  // namespace
 
 size_t attend_smem_bytes(int nheads, int batch) { return SmemLayout::total(nheads, batch); }
@@ -260,33 +192,25 @@ __global__ void __launch_bounds__(kAttendThreads, kAttendCtasPerSm) attend_kerne
   float* sComb = reinterpret_cast<float*>(smem + SmemLayout::comb_off);
   long long* sOff = reinterpret_cast<long long*>(smem + SmemLayout::hoff_off);
   int* sSeq = reinterpret_cast<int*>(smem + SmemLayout::seq_off(nheads));
-  __shared__ int is_last;
-  __shared__ const float* msrc[kMaxMerge];
-  __shared__ float mM[kMaxMerge][kMaxGroup];
-  __shared__ float mF[kMaxMerge][kMaxGroup];
-  __shared__ float mL[kMaxGroup];
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   pdl_wait();
 
   // ---- the layer's heads and their token-set lengths --------------------------------------
-  for (int b = tid; b < a.B; b += kAttendThreads) {
-    const int n = a.seq_lens[b];
-    sSeq[b] = n < 1 ? 1 : (n > a.max_ctx ? a.max_ctx : n);
-  }
-  __syncthreads();
   for (int hd = tid; hd < nheads; hd += kAttendThreads) {
     const int b = hd / a.Hkv, kvh = hd - b * a.Hkv;
-    const int N = sSeq[b];
-    int len;
     const bool ret = !a.dense && a.slot_of_kvh[kvh] >= 0;
+    const int n = a.seq_lens[b];  // both loads in flight together
+    const int ns = ret ? __ldcg(w.sel_total + b * a.nret + a.slot_of_kvh[kvh]) : 0;
+    const int N = n < 1 ? 1 : (n > a.max_ctx ? a.max_ctx : n);
+    if (kvh == 0) sSeq[b] = N;
+    int len;
     if ((a.heads == kHeadsLocal && ret) || (a.heads == kHeadsRetrieval && !ret)) {
       len = 0;  // another launch of this layer covers the head
     } else if (a.dense) {
       len = N;
     } else if (ret) {
-      len = __ldcg(w.sel_total + b * a.nret + a.slot_of_kvh[kvh]);
-      len = len < 1 ? 1 : (len > N ? N : len);
+      len = ns < 1 ? 1 : (ns > N ? N : ns);
     } else {
       len = window_len(N, a.window, a.sinks);
     }
@@ -309,10 +233,12 @@ __global__ void __launch_bounds__(kAttendThreads, kAttendCtasPerSm) attend_kerne
     if (lane == 0) sOff[0] = 0;
   }
   __syncthreads();
+  if (blockIdx.x == 0)  // merge_kernel finds the pieces of each head from these
+    for (int i = tid; i <= nheads; i += kAttendThreads) w.head_off[i] = sOff[i];
   pdl_launch_dependents();
 
   // P = min(grid, T) CTAs take part, so every range is non-empty and the pieces of a head are
-  // exactly the CTAs c_first..c_last (the ticket count of its merge)
+  // exactly the CTAs c_first..c_last
   const long long T = sOff[nheads];
   const long long P = min((long long)gridDim.x, T);  // T >= 1: the launch covers >= 1 head
   if ((long long)blockIdx.x >= P) return;
@@ -535,63 +461,116 @@ __global__ void __launch_bounds__(kAttendThreads, kAttendCtasPerSm) attend_kerne
       }
     }
     if (a.sel_count && (int)blockIdx.x == c_first && tid == 0) a.sel_count[hd] = (int)(he - hb);
-    if (!single) {
-      // Two-level merge tree over the pieces of this head, fan-in kMergeFanIn: the last CTA of
-      // each aligned group of kMergeFanIn CTAs merges the group's pieces, the last group merges
-      // the groups. Tickets only: nothing waits.
-      const int gi = (int)blockIdx.x / kMergeFanIn;
-      const int g_first = c_first / kMergeFanIn, g_last = c_last / kMergeFanIn;
-      const int gs = max(c_first, gi * kMergeFanIn);
-      const int ge = min(c_last, gi * kMergeFanIn + kMergeFanIn - 1);
-      bool holds_group = true;
-      if (ge > gs) {
-        __syncthreads();  // the piece is written (CTA scope); thread 0 publishes it (gpu scope)
-        unsigned* tk = w.ticket_group + (size_t)hd * w.n_merge_groups + gi;
-        if (tid == 0) {
-          __threadfence();
-          is_last = (atomicAdd(tk, 1u) == (unsigned)(ge - gs));
-          if (is_last) __threadfence();
-        }
-        __syncthreads();
-        holds_group = is_last;
-        if (holds_group) {
-          if (tid < ge - gs + 1)
-            msrc[tid] = w.partials + ((size_t)(gs + tid) + hd) * kPartFloats;
-          const bool final_merge = (g_first == g_last);
-          float* dst = final_merge ? out_h
-                                   : w.group_partials +
-                                         ((size_t)hd * w.n_merge_groups + gi) * kPartFloats;
-          merge_partials(ge - gs + 1, a.G, final_merge, dst, msrc, mM, mF, mL, tid);
-          if (tid == 0) *tk = 0u;
-          if (final_merge) holds_group = false;
-        }
-      }
-      if (holds_group) {  // this CTA holds group gi's merged result: join the head's merge
-        __syncthreads();
-        if (tid == 0) {
-          __threadfence();
-          is_last = (atomicAdd(w.ticket_attend + hd, 1u) == (unsigned)(g_last - g_first));
-          if (is_last) __threadfence();
-        }
-        __syncthreads();
-        if (is_last) {
-          const int ng = g_last - g_first + 1;
-          if (tid < ng) {
-            const int gg = g_first + tid;
-            const int s0 = max(c_first, gg * kMergeFanIn);
-            const int s1 = min(c_last, gg * kMergeFanIn + kMergeFanIn - 1);
-            msrc[tid] = (s1 > s0) ? w.group_partials + ((size_t)hd * w.n_merge_groups + gg) *
-                                                           kPartFloats
-                                  : w.partials + ((size_t)s0 + hd) * kPartFloats;
-          }
-          merge_partials(ng, a.G, true, out_h, msrc, mM, mF, mL, tid);
-          if (tid == 0) w.ticket_attend[hd] = 0u;
-        }
-      }
-    }
     __syncthreads();  // sComb is reused by the next piece
   }
   cp_async_wait<0>();  // nothing may land in shared memory after the CTA exits
+}
+
+// Combines the pieces of every head that the attention launch split over several CTAs.
+// Unit u = (head hd, query head jq of the group, quarter qtr of the 128 dimensions); one CTA of
+// kMergeThreads threads per unit. With M = max_i m_i and f_i = 2^(m_i - M) over the pieces
+// i = 0 .. n-1 of the head (in CTA order):  out[jq][d] = sum_i f_i O_i[jq][d] / sum_i f_i l_i.
+// Every sum runs in a fixed order (per-thread strides, then fixed shuffle and shared-memory
+// trees), so the result does not depend on timing. The first kMergeRows * kMergeRegs pieces'
+// O rows are loaded before the maxima are known, so m, l and O arrive in one round trip.
+__global__ void __launch_bounds__(kMergeThreads) merge_kernel(const LayerArgs a,
+                                                              const Workspace w,
+                                                              int attend_grid) {
+  __shared__ float sF[kMaxPieces];  // m_i, then the factor f_i
+  __shared__ float sL[kMaxPieces];
+  __shared__ float red[kMergeThreads / 32];
+  __shared__ float4 racc[kMergeThreads / 32][8];
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int r = tid >> 3, c = tid & 7;  // piece row, 16-byte column of the 32-dim quarter
+  const int nheads = a.B * a.Hkv;
+  const int units = merge_units(nheads, a.G);
+  pdl_wait();
+  pdl_launch_dependents();
+  const long long T = __ldcg(w.head_off + nheads);
+  const long long P = min((long long)attend_grid, T);
+  for (int u = blockIdx.x; u < units; u += gridDim.x) {
+    const int hd = u / (a.G * 4), jq = (u >> 2) % a.G, qtr = u & 3;
+    const long long hb = __ldcg(w.head_off + hd), he = __ldcg(w.head_off + hd + 1);
+    if (he <= hb) continue;
+    const int c_first = (int)cta_of(hb, T, P), c_last = (int)cta_of(he - 1, T, P);
+    if (c_first == c_last) continue;  // written by the attention launch
+    const int n = c_last - c_first + 1;
+    const float* base = w.partials + (size_t)(c_first + hd) * kPartFloats;
+    const int col = jq * kHeadDim + qtr * 32 + c * 4;
+    float4 ov[kMergeRegs];
+#pragma unroll
+    for (int k = 0; k < kMergeRegs; ++k) {
+      const int i = r + k * kMergeRows;
+      ov[k] = (i < n) ? __ldcg(reinterpret_cast<const float4*>(base + (size_t)i * kPartFloats + col))
+                      : make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+    float mx = -INFINITY;
+    for (int i = tid; i < n; i += kMergeThreads) {
+      const float m = __ldcg(base + (size_t)i * kPartFloats + kPartO + jq);
+      sL[i] = __ldcg(base + (size_t)i * kPartFloats + kPartO + kMaxGroup + jq);
+      sF[i] = m;
+      mx = fmaxf(mx, m);
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+    if (lane == 0) red[warp] = mx;
+    __syncthreads();
+    float M = red[0];
+#pragma unroll
+    for (int k = 1; k < kMergeThreads / 32; ++k) M = fmaxf(M, red[k]);
+    float ls = 0.f;
+    for (int i = tid; i < n; i += kMergeThreads) {
+      const float f = exp2f(sF[i] - M);
+      sF[i] = f;
+      ls += sL[i] * f;
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) ls += __shfl_xor_sync(0xffffffffu, ls, o);
+    __syncthreads();  // every thread has read red[] (the maxima)
+    if (lane == 0) red[warp] = ls;
+    __syncthreads();  // red[] holds the l sums, sF[] the factors
+    float L = 0.f;
+#pragma unroll
+    for (int k = 0; k < kMergeThreads / 32; ++k) L += red[k];
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+    for (int k = 0; k < kMergeRegs; ++k) {
+      const int i = r + k * kMergeRows;
+      if (i < n) {
+        const float f = sF[i];
+        acc.x += ov[k].x * f; acc.y += ov[k].y * f; acc.z += ov[k].z * f; acc.w += ov[k].w * f;
+      }
+    }
+    for (int i = r + kMergeRegs * kMergeRows; i < n; i += kMergeRows) {  // long heads only
+      const float4 v = __ldcg(reinterpret_cast<const float4*>(base + (size_t)i * kPartFloats + col));
+      const float f = sF[i];
+      acc.x += v.x * f; acc.y += v.y * f; acc.z += v.z * f; acc.w += v.w * f;
+    }
+    // rows r of a warp: (tid >> 3) & 3; add them (lanes c, c + 8, c + 16, c + 24), then warps
+#pragma unroll
+    for (int o = 8; o < 32; o <<= 1) {
+      acc.x += __shfl_xor_sync(0xffffffffu, acc.x, o);
+      acc.y += __shfl_xor_sync(0xffffffffu, acc.y, o);
+      acc.z += __shfl_xor_sync(0xffffffffu, acc.z, o);
+      acc.w += __shfl_xor_sync(0xffffffffu, acc.w, o);
+    }
+    if (lane < 8) racc[warp][lane] = acc;
+    __syncthreads();
+    if (tid < 8) {
+      float4 o = racc[0][tid];
+#pragma unroll
+      for (int k = 1; k < kMergeThreads / 32; ++k) {
+        const float4 v = racc[k][tid];
+        o.x += v.x; o.y += v.y; o.z += v.z; o.w += v.w;
+      }
+      const float inv = 1.f / L;
+      const int b = hd / a.Hkv, kvh = hd - b * a.Hkv;
+      float4* dst = reinterpret_cast<float4*>(
+          a.out + ((size_t)b * a.Hq + (size_t)kvh * a.G + jq) * kHeadDim + qtr * 32 + tid * 4);
+      *dst = make_float4(o.x * inv, o.y * inv, o.z * inv, o.w * inv);
+    }
+    __syncthreads();  // shared arrays are reused by the next unit
+  }
 }
 
 }  // namespace rtp

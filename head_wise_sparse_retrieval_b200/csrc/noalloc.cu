@@ -2,8 +2,8 @@
 //
 // For callers that cannot allocate device memory (a serving engine that owns every byte
 // through its own pool, or a latency-critical path where cudaMalloc, which may synchronise the
-// device, must not run). The attention kernel's only scratch -- split-K partials, merged group
-// partials, merge tickets and a status word -- lives in the file-scope device array below, of
+// device, must not run). The attention kernels' only scratch -- split-K partials, the head
+// offsets the merge reads and a status word -- lives in the file-scope device array below, of
 // a fixed size that bounds the call (at most RTP_NOALLOC_MAX_HEADS KV heads per call and at most
 // RTP_NOALLOC_MAX_CTAS attention CTAs). Host code never touches the array by name: its device
 // address is looked up once per device with cudaGetSymbolAddress and passed to the kernel.
@@ -21,16 +21,14 @@ namespace {
 
 constexpr int kNaHeads = RTP_NOALLOC_MAX_HEADS;
 constexpr int kNaCtas = RTP_NOALLOC_MAX_CTAS;
-constexpr int kNaGroups = (kNaCtas + kMergeFanIn - 1) / kMergeFanIn;
 constexpr size_t kNaPartOff = 0;
 constexpr size_t kNaPartBytes = (size_t)(kNaCtas + kNaHeads) * kPartFloats * 4;
-constexpr size_t kNaGroupOff = kNaPartOff + kNaPartBytes;
-constexpr size_t kNaGroupBytes = (size_t)kNaHeads * kNaGroups * kPartFloats * 4;
-constexpr size_t kNaTicketOff = kNaGroupOff + kNaGroupBytes;       // attend tickets, then group
-constexpr size_t kNaTicketBytes = ((size_t)kNaHeads * (1 + kNaGroups) + 64) * 4;  // + status
-constexpr size_t kNaUsed = kNaTicketOff + kNaTicketBytes;
+constexpr size_t kNaHeadOff = kNaPartOff + kNaPartBytes;           // head offsets, then status
+constexpr size_t kNaStatusOff = kNaHeadOff + ((size_t)kNaHeads + 1) * 8;
+constexpr size_t kNaUsed = kNaStatusOff + 256;
 static_assert(kNaUsed <= RTP_NOALLOC_SCRATCH_BYTES, "no-alloc scratch too small");
-static_assert(kNaCtas <= 2 * kMergeFanIn * kMergeFanIn, "two merge levels cover the grid");
+static_assert(kNaCtas <= kMaxPieces, "the merge holds one factor per attention CTA");
+static_assert(kNaHeadOff % 256 == 0, "aligned head offsets");
 
 // The scratch of every rtp_window_attention_noalloc call on this device.
 static __device__ __align__(256) unsigned char g_noalloc_scratch[RTP_NOALLOC_SCRATCH_BYTES];
@@ -129,22 +127,20 @@ extern "C" rtp_status rtp_window_attention_noalloc(const rtp_noalloc_params* p, 
   memset(&w, 0, sizeof w);
   unsigned char* base = setup.scratch;
   w.partials = reinterpret_cast<float*>(base + kNaPartOff);
-  w.group_partials = reinterpret_cast<float*>(base + kNaGroupOff);
-  w.ticket_attend = reinterpret_cast<unsigned*>(base + kNaTicketOff);
-  w.ticket_group = w.ticket_attend + kNaHeads;
-  w.status = w.ticket_group + (size_t)kNaHeads * kNaGroups;
-  w.n_merge_groups = kNaGroups;
+  w.head_off = reinterpret_cast<long long*>(base + kNaHeadOff);
+  w.status = reinterpret_cast<unsigned*>(base + kNaStatusOff);
 
+  // Nothing in the array needs to start at zero: the attention launch writes the head offsets
+  // and every partial the merge reads; status bits only accumulate.
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  // the tickets must start at zero whatever the previous call left behind
-  e = cudaMemsetAsync(base + kNaTicketOff, 0, kNaTicketBytes, s);
-  if (e != cudaSuccess) return na_fail(RTP_ERR_CUDA, "cannot clear the merge tickets");
-
   int grid = setup.num_sms * kAttendCtasPerSm;
   if (grid > kNaCtas) grid = kNaCtas;
   attend_kernel<<<grid, kAttendThreads, smem, s>>>(a, w);
   e = cudaGetLastError();
   if (e != cudaSuccess) return na_fail(RTP_ERR_CUDA, "attention kernel launch failed");
+  merge_kernel<<<merge_units(nheads, a.G), kMergeThreads, 0, s>>>(a, w, grid);
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return na_fail(RTP_ERR_CUDA, "merge kernel launch failed");
   set_last_error("");
   return RTP_OK;
 }

@@ -105,7 +105,6 @@ struct WsPlan {
 WsPlan plan_workspace(const rtp_config* c, int attend_grid, int select_grid) {
   const size_t slots = (size_t)c->batch * c->num_kv_heads;
   const size_t nmax = round_up((size_t)c->max_ctx, 64);  // per-slot stride (16-byte loads)
-  const size_t ngroups = ((size_t)attend_grid + kMergeFanIn - 1) / kMergeFanIn;
   const size_t sizes[] = {
       slots * nmax * 4,                      // 0 scores
       slots * (size_t)select_grid * 4,       // 1 cta_max
@@ -120,11 +119,9 @@ WsPlan plan_workspace(const rtp_config* c, int attend_grid, int select_grid) {
       slots * 4,                             // 10 sel_n
       (size_t)(2 + (4 * kMaxAttendHeads + 15) / 16) * 4,  // 11 grid_bar
       4,                                     // 12 (unused)
-      slots * 4,                             // 13 ticket_attend
+      (slots + 1) * 8,                       // 13 head_off
       ((size_t)attend_grid + slots) * kPartFloats * 4,  // 14 partials
       256,                                   // 15 status
-      slots * ngroups * 4,                   // 16 ticket_group
-      slots * ngroups * kPartFloats * 4,  // 17 group_partials
   };
   WsPlan p{};
   size_t at = 0;
@@ -136,9 +133,9 @@ WsPlan plan_workspace(const rtp_config* c, int attend_grid, int select_grid) {
   return p;
 }
 
-template <typename Kernel>
+template <typename Kernel, typename... Args>
 cudaError_t launch_pdl(Kernel k, dim3 grid, dim3 block, size_t smem, cudaStream_t s,
-                       const LayerArgs& a, const Workspace& w, bool cooperative) {
+                       bool cooperative, Args... args) {
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = grid;
   cfg.blockDim = block;
@@ -151,7 +148,7 @@ cudaError_t launch_pdl(Kernel k, dim3 grid, dim3 block, size_t smem, cudaStream_
   attr[1].val.cooperative = 1;
   cfg.attrs = attr;
   cfg.numAttrs = cooperative ? 2 : 1;
-  return cudaLaunchKernelEx(&cfg, k, a, w);
+  return cudaLaunchKernelEx(&cfg, k, args...);
 }
 
 rtp_status check_io(const rtp_handle* h, const rtp_layer_io* io, bool need_idx) {
@@ -204,14 +201,13 @@ LayerArgs make_args(const rtp_handle* h, const rtp_layer_io* io) {
 constexpr int kProfCapacity = 1024;
 
 // Launches one kernel, bracketed by profiling events when the handle has profiling enabled.
-template <typename Kernel>
+template <typename Kernel, typename... Args>
 cudaError_t launch_one(rtp_handle* h, int kind, Kernel k, dim3 grid, dim3 block, size_t smem,
-                       cudaStream_t s, const LayerArgs& a, const Workspace& ws,
-                       bool cooperative = false) {
+                       cudaStream_t s, bool cooperative, Args... args) {
   const bool prof = h->prof && h->prof_used < kProfCapacity;
   if (h->prof && !prof) h->prof_overflow = true;
   if (prof) cudaEventRecord(h->prof_ev[2 * h->prof_used], s);
-  cudaError_t e = launch_pdl(k, grid, block, smem, s, a, ws, cooperative);
+  cudaError_t e = launch_pdl(k, grid, block, smem, s, cooperative, args...);
   if (prof && e == cudaSuccess) {
     cudaEventRecord(h->prof_ev[2 * h->prof_used + 1], s);
     h->prof_kind[h->prof_used++] = kind;
@@ -223,14 +219,17 @@ rtp_status enqueue_layer(rtp_handle* h, const LayerArgs& a0, cudaStream_t s) {
   cudaError_t e;
   if (!a0.dense && a0.nret > 0) {
     e = launch_one(h, 0, select_kernel, dim3(h->select_grid), dim3(kSelThreads), h->select_smem,
-                   s, a0, h->ws, true);
+                   s, true, a0, h->ws);
     if (e != cudaSuccess) return cuda_fail(e, "select_kernel launch");
   }
   LayerArgs a = a0;
   a.heads = kHeadsAll;
   e = launch_one(h, 1, attend_kernel, dim3(h->attend_grid), dim3(kAttendThreads), h->attend_smem,
-                 s, a, h->ws);
-  return e == cudaSuccess ? RTP_OK : cuda_fail(e, "attend_kernel launch");
+                 s, false, a, h->ws);
+  if (e != cudaSuccess) return cuda_fail(e, "attend_kernel launch");
+  e = launch_one(h, 2, merge_kernel, dim3(merge_units(a.B * a.Hkv, a.G)), dim3(kMergeThreads),
+                 0, s, false, a, h->ws, h->attend_grid);
+  return e == cudaSuccess ? RTP_OK : cuda_fail(e, "merge_kernel launch");
 }
 
 struct DeviceGuard {
@@ -298,7 +297,7 @@ rtp_status rtp_create(const rtp_config* cfg, int device, rtp_handle** out) {
   h->G = cfg->num_q_heads / cfg->num_kv_heads;
   cudaDeviceGetAttribute(&h->num_sms, cudaDevAttrMultiProcessorCount, device);
   h->attend_grid = h->num_sms * kAttendCtasPerSm;  // persistent: every CTA resident
-  if (h->attend_grid > 2 * kMergeFanIn * kMergeFanIn) h->attend_grid = 2 * kMergeFanIn * kMergeFanIn;
+  if (h->attend_grid > kMaxPieces) h->attend_grid = kMaxPieces;
 
   h->select_smem = select_smem_bytes(cfg->batch * cfg->num_kv_heads);
   e = cudaFuncSetAttribute(select_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -351,12 +350,9 @@ rtp_status rtp_create(const rtp_config* cfg, int device, rtp_handle** out) {
   w.sel_total = reinterpret_cast<int*>(base + p.off[9]);
   w.sel_n = reinterpret_cast<int*>(base + p.off[10]);
   w.grid_bar = reinterpret_cast<unsigned*>(base + p.off[11]);
-  w.ticket_attend = reinterpret_cast<unsigned*>(base + p.off[13]);
+  w.head_off = reinterpret_cast<long long*>(base + p.off[13]);
   w.partials = reinterpret_cast<float*>(base + p.off[14]);
   w.status = reinterpret_cast<unsigned*>(base + p.off[15]);
-  w.ticket_group = reinterpret_cast<unsigned*>(base + p.off[16]);
-  w.group_partials = reinterpret_cast<float*>(base + p.off[17]);
-  w.n_merge_groups = (h->attend_grid + kMergeFanIn - 1) / kMergeFanIn;
   w.ld = (int)round_up((size_t)cfg->max_ctx, 64);
   h->stage_q = base + stage_q_off;
   h->stage_qidx = base + stage_qi_off;

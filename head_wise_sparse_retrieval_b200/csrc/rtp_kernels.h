@@ -24,13 +24,10 @@ struct Workspace {
   int* sel_total;                 // [slots]                 |S|
   int* sel_n;                     // [slots]                 N the selection was made over
   unsigned* grid_bar;             // grid barrier of the selection kernel: generation, root, groups
-  unsigned* ticket_attend;        // [B*Hkv]                 merge of a head's groups
-  unsigned* ticket_group;         // [B*Hkv][n_merge_groups] merge of a group's pieces
-  float* partials;                // [(attend_ctas + B*Hkv)][kPartFloats]  one per piece
-  float* group_partials;          // [B*Hkv][n_merge_groups][kPartFloats]
+  float* partials;                // [(attend_ctas + B*Hkv)][kPartFloats]  piece of CTA c, head h at c + h
+  long long* head_off;            // [B*Hkv + 1]             prefix sums of the heads' token-set sizes
   unsigned* status;               // [1] RTP_DEV_* bits
   int ld;                         // per-slot stride of scores / sel_idx: max_ctx rounded up to 64
-  int n_merge_groups;             // ceil(attend_ctas / kMergeFanIn)
 };
 
 struct LayerArgs {
@@ -55,6 +52,7 @@ enum : int { kHeadsAll = 0, kHeadsLocal = 1, kHeadsRetrieval = 2 };
 // Kernel entry points (defined in select_kernels.cu / attend_kernel.cu).
 __global__ void select_kernel(const LayerArgs a, const Workspace w);  // cooperative launch
 __global__ void attend_kernel(const LayerArgs a, const Workspace w);
+__global__ void merge_kernel(const LayerArgs a, const Workspace w, int attend_grid);
 
 constexpr int kAttendWarps = 4;                          // warps per attention CTA
 constexpr int kAttendDepth = 3;                          // cp.async stages per warp
@@ -66,8 +64,10 @@ constexpr int kMaxSelSlots = kMaxAttendHeads;            // retrieval slots per 
 constexpr int kMaxSelectCtasPerSm = 2;                   // resident selection CTAs per SM
 constexpr int kScoreCap = 16384;                         // scores a selection CTA keeps on chip
 size_t select_smem_bytes(int slots);
-constexpr int kMergeFanIn = 16;                          // pieces merged per tree node
-// the attention grid is at most kMergeFanIn * 2 * kMergeFanIn CTAs (two merge levels)
+constexpr int kMaxPieces = 1024;                         // attention CTAs (pieces of one head)
+constexpr int kMergeThreads = 128;
+// merge units: (head, query head of the group, quarter of the 128 dimensions)
+__host__ __device__ inline int merge_units(int nheads, int G) { return nheads * G * 4; }
 
 size_t attend_smem_bytes(int nheads, int batch);
 void set_last_error(const char* msg);  // the reason rtp_last_error reports on this thread

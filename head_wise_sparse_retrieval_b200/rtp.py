@@ -26,7 +26,7 @@ EXPORTS = ("rtp_config_default", "rtp_workspace_bytes", "rtp_create", "rtp_destr
            "rtp_get_threshold", "rtp_get_device_status", "rtp_status_string", "rtp_last_error",
            "rtp_profile_enable", "rtp_profile_read", "rtp_window_attention_noalloc")
 NOALLOC_MAX_HEADS = 64
-KERNEL_CLASSES = ("select", "attend", "reserved2", "reserved3")
+KERNEL_CLASSES = ("select", "attend", "merge", "reserved3")
 
 
 class RtpError(RuntimeError):

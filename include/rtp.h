@@ -162,7 +162,7 @@ RTP_API rtp_status rtp_get_threshold(rtp_handle *h, int b, int kvh, int *bstar, 
  * launches on this handle is bracketed by two CUDA events recorded on the launch stream (the
  * events are created here, so the decode calls still allocate nothing). Do not enable it while
  * capturing a CUDA graph. Kernel classes: 0 selection (indexer score, histogram top-p,
- * compaction), 1 attention; 2 and 3 are reserved (always 0). The event pool holds 1024
+ * compaction), 1 attention, 2 merge of split heads' partials; 3 is reserved (always 0). The event pool holds 1024
  * launches; rtp_profile_read empties it. Errors: RTP_ERR_CUDA if the events cannot be created. */
 RTP_API rtp_status rtp_profile_enable(rtp_handle *h, int enable);
 
@@ -179,7 +179,7 @@ RTP_API rtp_status rtp_get_device_status(rtp_handle *h, uint32_t *code);
  * engines that plan every byte up front and hand out memory only from their own pool, and
  * latency-critical paths where cudaMalloc (which may synchronise the device) must not run.
  * rtp_create allocates a workspace; this entry point needs no handle: its only scratch (the
- * split-K partials and merge tickets of the attention kernel) is a file-scope device array of
+ * split-K partials and head offsets of the attention kernels) is a file-scope device array of
  * RTP_NOALLOC_SCRATCH_BYTES that every GPU loading the library holds until the process exits.
  *
  * It computes, for every (b, KV head), the attention over the window + sink set of a local
@@ -193,7 +193,7 @@ RTP_API rtp_status rtp_get_device_status(rtp_handle *h, uint32_t *code);
  * It calls no cudaMalloc / cudaFree and no allocating library routine. The first call on a
  * device looks up the array's device address (cudaGetSymbolAddress) with that device current;
  * make that first call before any stream capture. Every call shares the one array, which keeps
- * the last call's contents; the call clears the tickets it needs (an async memset on `stream`).
+ * the last call's contents, none of which a later call reads before writing it.
  * Calls that overlap on the GPU (different streams, or the same array used from two threads'
  * streams at once) race on the array. Device-side problems (a seq_lens entry outside
  * [1, max_ctx], which is clamped) are not reported by this call. */
