@@ -10,8 +10,8 @@
 // set; dense mode: all N) and the concatenation is cut into P equal ranges, one per CTA
 // (split-K, balanced to the token). A CTA cuts its range, head by head, into 16-token tiles
 // dealt round-robin to its warps. Each warp runs its own kAttendDepth-deep pipeline:
-//   * positions: the selected list (prefetched one tile ahead, so the load overlaps the
-//     math) or window arithmetic;
+//   * positions: the selected list, loaded two tiles before the tile's data is requested (the
+//     index round trip overlaps two tiles of streaming), or window arithmetic;
 //   * data: each tile's 16 K rows and 16 V rows (256 B each) are gathered with 16-byte
 //     cp.async (L2 evict-first; rows past the end of a head are zero-filled, not read);
 //   * math on the tensor cores (mma m16n8k16, bf16 in, fp32 accumulate) with the 8 query
@@ -60,11 +60,6 @@ __device__ __forceinline__ int window_len(int N, int W, int S) {
 }
 __device__ __forceinline__ int window_pos(int r, int N, int W, int S) {
   return (N <= W + S) ? r : (r < S ? r : N - W + (r - S));
-}
-
-// CTA whose range [floor(c T / P), floor((c+1) T / P)) holds position x (0 <= x < T, P <= T).
-__device__ __forceinline__ long long cta_of(long long x, long long T, long long P) {
-  return ((x + 1) * P + T - 1) / T - 1;
 }
 
 // The segments of this CTA's range, head by head, in order.
@@ -205,9 +200,7 @@ __global__ void __launch_bounds__(kAttendThreads, kAttendCtasPerSm) attend_kerne
     const int N = n < 1 ? 1 : (n > a.max_ctx ? a.max_ctx : n);
     if (kvh == 0) sSeq[b] = N;
     int len;
-    if ((a.heads == kHeadsLocal && ret) || (a.heads == kHeadsRetrieval && !ret)) {
-      len = 0;  // another launch of this layer covers the head
-    } else if (a.dense) {
+    if (a.dense) {
       len = N;
     } else if (ret) {
       len = ns < 1 ? 1 : (ns > N ? N : ns);
@@ -233,8 +226,6 @@ __global__ void __launch_bounds__(kAttendThreads, kAttendCtasPerSm) attend_kerne
     if (lane == 0) sOff[0] = 0;
   }
   __syncthreads();
-  if (blockIdx.x == 0)  // merge_kernel finds the pieces of each head from these
-    for (int i = tid; i <= nheads; i += kAttendThreads) w.head_off[i] = sOff[i];
   pdl_launch_dependents();
 
   // P = min(grid, T) CTAs take part, so every range is non-empty and the pieces of a head are
@@ -242,8 +233,8 @@ __global__ void __launch_bounds__(kAttendThreads, kAttendCtasPerSm) attend_kerne
   const long long T = sOff[nheads];
   const long long P = min((long long)gridDim.x, T);  // T >= 1: the launch covers >= 1 head
   if ((long long)blockIdx.x >= P) return;
-  const long long t0 = (long long)blockIdx.x * T / P;
-  const long long t1 = ((long long)blockIdx.x + 1) * T / P;
+  const long long t0 = floor_div((long long)blockIdx.x * T, P);
+  const long long t1 = floor_div(((long long)blockIdx.x + 1) * T, P);
 
   // total tiles of this CTA (segments are few)
   int ktot = 0;
@@ -260,33 +251,50 @@ __global__ void __launch_bounds__(kAttendThreads, kAttendCtasPerSm) attend_kerne
   // ---- load side: this warp's tiles k = warp + kWarps i, positions one tile ahead ----------
   TileIter iss;
   iss.begin(sOff, nheads, t0, t1);
-  HeadRef pf_h{};
-  int pf_r = 0, pf_n = 0, pf_pos = -1, pf_hd = -1;
-  auto prefetch = [&](int i) {  // positions of warp tile i (pf_n = 0 past the end)
+  // Two position slots: A holds the next tile to issue, B the one after. fill() loads a tile's
+  // positions into B; issue() requests the data of A's tile, then A takes B.
+  HeadRef fill_h{}, iss_h{};
+  int fill_hd = -1, iss_hd = -1;
+  int a_hd = -1, a_n = 0, a_pos = -1, b_hd = -1, b_n = 0, b_pos = -1;
+  auto fill = [&](int i) {  // positions of warp tile i into B (b_n = 0 past the end)
     const int k = warp + kWarps * i;
-    pf_n = 0;
-    pf_pos = -1;
+    b_n = 0;
+    b_pos = -1;
     if (k < ktot && iss.locate(k)) {
-      if (iss.hd != pf_hd) {
-        pf_hd = iss.hd;
-        pf_h = head_ref(a, w, sSeq, pf_hd);
+      if (iss.hd != fill_hd) {
+        fill_hd = iss.hd;
+        fill_h = head_ref(a, w, sSeq, fill_hd);
       }
-      pf_r = iss.r0 + (k - iss.kb) * kTile;
-      pf_n = min(kTile, iss.r1 - pf_r);
-      pf_pos = tile_positions(pf_h, a, pf_r, pf_n, lane);
+      const int r = iss.r0 + (k - iss.kb) * kTile;
+      b_hd = fill_hd;
+      b_n = min(kTile, iss.r1 - r);
+      b_pos = tile_positions(fill_h, a, r, b_n, lane);
     }
   };
-  auto issue = [&](int i) {  // loads of warp tile i (positions prefetched); one commit group
-    if (pf_n > 0)
-      issue_tile(my_stages + (i % kDepth) * kWarpStage, pf_h, pf_pos, pf_n, lane, policy,
+  auto shift = [&]() {
+    a_hd = b_hd;
+    a_n = b_n;
+    a_pos = b_pos;
+  };
+  auto issue = [&](int i) {  // loads of warp tile i (A's positions); one commit group
+    if (a_n > 0) {
+      if (a_hd != iss_hd) {
+        iss_hd = a_hd;
+        iss_h = head_ref(a, w, sSeq, iss_hd);
+      }
+      issue_tile(my_stages + (i % kDepth) * kWarpStage, iss_h, a_pos, a_n, lane, policy,
                  w.status);
+    }
     cp_async_commit();
   };
   for (int s = 0; s < kDepth - 1; ++s) {
-    prefetch(s);
+    fill(s);
+    shift();
     issue(s);
   }
-  prefetch(kDepth - 1);
+  fill(kDepth - 1);
+  shift();
+  fill(kDepth);
 
   // ---- math side: segment by segment ----
   const int g = lane >> 2, t = lane & 3;  // MMA fragment coordinates
@@ -323,7 +331,8 @@ __global__ void __launch_bounds__(kAttendThreads, kAttendCtasPerSm) attend_kerne
       // keep kDepth - 1 tiles in flight: issue warp tile done + kDepth - 1, then prefetch the
       // positions of the one after (their load overlaps this tile's math)
       issue(done + kDepth - 1);
-      prefetch(done + kDepth);
+      shift();
+      fill(done + kDepth + 1);
       cp_async_wait<kDepth - 1>();
       __syncwarp();
 
@@ -433,11 +442,13 @@ __global__ void __launch_bounds__(kAttendThreads, kAttendCtasPerSm) attend_kerne
       }
     }
 
-    const long long hb = sOff[hd], he = sOff[hd + 1];
-    const int c_first = (int)cta_of(hb, T, P), c_last = (int)cta_of(he - 1, T, P);
+    // this CTA holds the head's first piece when its segment starts at rank 0, the last when
+    // it ends at the head's size; one piece covering both is the whole head
+    const int len = (int)(sOff[hd + 1] - sOff[hd]);
+    const bool first_piece = (r0 == 0), last_piece = (r1 == len);
     const int d = tid;  // 0..127: one output dimension per thread
     float* out_h = a.out + ((size_t)b * a.Hq + (size_t)kvh * a.G) * kHeadDim;
-    const bool single = (c_first == c_last);
+    const bool single = first_piece && last_piece;
     float* piece = w.partials + ((size_t)blockIdx.x + hd) * kPartFloats;
     for (int jq = 0; jq < a.G; ++jq) {
       float M = -INFINITY;
@@ -460,7 +471,11 @@ __global__ void __launch_bounds__(kAttendThreads, kAttendCtasPerSm) attend_kerne
         }
       }
     }
-    if (a.sel_count && (int)blockIdx.x == c_first && tid == 0) a.sel_count[hd] = (int)(he - hb);
+    if (tid == 0) {  // merge_kernel reads the head's piece range (CTAs first .. last)
+      if (first_piece) w.head_pieces[hd].x = (int)blockIdx.x;
+      if (last_piece) w.head_pieces[hd].y = (int)blockIdx.x;
+      if (a.sel_count && first_piece) a.sel_count[hd] = len;
+    }
     __syncthreads();  // sComb is reused by the next piece
   }
   cp_async_wait<0>();  // nothing may land in shared memory after the CTA exits
@@ -474,8 +489,7 @@ __global__ void __launch_bounds__(kAttendThreads, kAttendCtasPerSm) attend_kerne
 // trees), so the result does not depend on timing. The first kMergeRows * kMergeRegs pieces'
 // O rows are loaded before the maxima are known, so m, l and O arrive in one round trip.
 __global__ void __launch_bounds__(kMergeThreads) merge_kernel(const LayerArgs a,
-                                                              const Workspace w,
-                                                              int attend_grid) {
+                                                              const Workspace w) {
   __shared__ float sF[kMaxPieces];  // m_i, then the factor f_i
   __shared__ float sL[kMaxPieces];
   __shared__ float red[kMergeThreads / 32];
@@ -486,15 +500,11 @@ __global__ void __launch_bounds__(kMergeThreads) merge_kernel(const LayerArgs a,
   const int units = merge_units(nheads, a.G);
   pdl_wait();
   pdl_launch_dependents();
-  const long long T = __ldcg(w.head_off + nheads);
-  const long long P = min((long long)attend_grid, T);
   for (int u = blockIdx.x; u < units; u += gridDim.x) {
     const int hd = u / (a.G * 4), jq = (u >> 2) % a.G, qtr = u & 3;
-    const long long hb = __ldcg(w.head_off + hd), he = __ldcg(w.head_off + hd + 1);
-    if (he <= hb) continue;
-    const int c_first = (int)cta_of(hb, T, P), c_last = (int)cta_of(he - 1, T, P);
-    if (c_first == c_last) continue;  // written by the attention launch
-    const int n = c_last - c_first + 1;
+    const int2 pr = __ldcg(w.head_pieces + hd);
+    const int c_first = pr.x, n = pr.y - pr.x + 1;
+    if (n <= 1) continue;  // written by the attention launch
     const float* base = w.partials + (size_t)(c_first + hd) * kPartFloats;
     const int col = jq * kHeadDim + qtr * 32 + c * 4;
     float4 ov[kMergeRegs];

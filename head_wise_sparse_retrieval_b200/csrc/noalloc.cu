@@ -2,8 +2,8 @@
 //
 // For callers that cannot allocate device memory (a serving engine that owns every byte
 // through its own pool, or a latency-critical path where cudaMalloc, which may synchronise the
-// device, must not run). The attention kernels' only scratch -- split-K partials, the head
-// offsets the merge reads and a status word -- lives in the file-scope device array below, of
+// device, must not run). The attention kernels' only scratch -- split-K partials, the piece
+// ranges the merge reads and a status word -- lives in the file-scope device array below, of
 // a fixed size that bounds the call (at most RTP_NOALLOC_MAX_HEADS KV heads per call and at most
 // RTP_NOALLOC_MAX_CTAS attention CTAs). Host code never touches the array by name: its device
 // address is looked up once per device with cudaGetSymbolAddress and passed to the kernel.
@@ -23,12 +23,12 @@ constexpr int kNaHeads = RTP_NOALLOC_MAX_HEADS;
 constexpr int kNaCtas = RTP_NOALLOC_MAX_CTAS;
 constexpr size_t kNaPartOff = 0;
 constexpr size_t kNaPartBytes = (size_t)(kNaCtas + kNaHeads) * kPartFloats * 4;
-constexpr size_t kNaHeadOff = kNaPartOff + kNaPartBytes;           // head offsets, then status
-constexpr size_t kNaStatusOff = kNaHeadOff + ((size_t)kNaHeads + 1) * 8;
+constexpr size_t kNaHeadOff = kNaPartOff + kNaPartBytes;           // piece ranges, then status
+constexpr size_t kNaStatusOff = kNaHeadOff + (size_t)kNaHeads * 8;
 constexpr size_t kNaUsed = kNaStatusOff + 256;
 static_assert(kNaUsed <= RTP_NOALLOC_SCRATCH_BYTES, "no-alloc scratch too small");
 static_assert(kNaCtas <= kMaxPieces, "the merge holds one factor per attention CTA");
-static_assert(kNaHeadOff % 256 == 0, "aligned head offsets");
+static_assert(kNaHeadOff % 256 == 0, "aligned piece ranges");
 
 // The scratch of every rtp_window_attention_noalloc call on this device.
 static __device__ __align__(256) unsigned char g_noalloc_scratch[RTP_NOALLOC_SCRATCH_BYTES];
@@ -119,7 +119,6 @@ extern "C" rtp_status rtp_window_attention_noalloc(const rtp_noalloc_params* p, 
   a.sinks = p->sinks;
   a.nret = 0;
   a.dense = p->dense ? 1 : 0;
-  a.heads = kHeadsAll;
   a.attn_scale_log2 = (float)((double)p->attn_scale * 1.4426950408889634);
   for (int k = 0; k < kMaxKvHeads; ++k) a.slot_of_kvh[k] = -1;
 
@@ -127,18 +126,18 @@ extern "C" rtp_status rtp_window_attention_noalloc(const rtp_noalloc_params* p, 
   memset(&w, 0, sizeof w);
   unsigned char* base = setup.scratch;
   w.partials = reinterpret_cast<float*>(base + kNaPartOff);
-  w.head_off = reinterpret_cast<long long*>(base + kNaHeadOff);
+  w.head_pieces = reinterpret_cast<int2*>(base + kNaHeadOff);
   w.status = reinterpret_cast<unsigned*>(base + kNaStatusOff);
 
-  // Nothing in the array needs to start at zero: the attention launch writes the head offsets
-  // and every partial the merge reads; status bits only accumulate.
+  // Nothing in the array needs to start at zero: the attention launch writes the piece range of
+  // every head and every partial the merge reads; status bits only accumulate.
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   int grid = setup.num_sms * kAttendCtasPerSm;
   if (grid > kNaCtas) grid = kNaCtas;
   attend_kernel<<<grid, kAttendThreads, smem, s>>>(a, w);
   e = cudaGetLastError();
   if (e != cudaSuccess) return na_fail(RTP_ERR_CUDA, "attention kernel launch failed");
-  merge_kernel<<<merge_units(nheads, a.G), kMergeThreads, 0, s>>>(a, w, grid);
+  merge_kernel<<<merge_units(nheads, a.G), kMergeThreads, 0, s>>>(a, w);
   e = cudaGetLastError();
   if (e != cudaSuccess) return na_fail(RTP_ERR_CUDA, "merge kernel launch failed");
   set_last_error("");

@@ -108,18 +108,18 @@ WsPlan plan_workspace(const rtp_config* c, int attend_grid, int select_grid) {
   const size_t sizes[] = {
       slots * nmax * 4,                      // 0 scores
       slots * (size_t)select_grid * 4,       // 1 cta_max
-      slots * kBins * 8,                     // 2 hist
+      (size_t)kHistCopies * slots * kBins * 8,  // 2 hist
       slots * 4,                             // 3 s_max
       slots * 4,                             // 4 bstar
       slots * 8,                             // 5 mass_total
       slots * nmax * 4,                      // 6 sel_idx
-      slots * (size_t)select_grid * kBins * 4,  // 7 cta_bins
-      4,                                     // 8 (unused)
+      slots * (size_t)select_grid * kBins * 4,  // 7 cta_ge
+      slots * nmax,                          // 8 bins
       slots * 4,                             // 9 sel_total
       slots * 4,                             // 10 sel_n
       (size_t)(2 + (4 * kMaxAttendHeads + 15) / 16) * 4,  // 11 grid_bar
       4,                                     // 12 (unused)
-      (slots + 1) * 8,                       // 13 head_off
+      slots * 8,                             // 13 head_pieces
       ((size_t)attend_grid + slots) * kPartFloats * 4,  // 14 partials
       256,                                   // 15 status
   };
@@ -218,17 +218,19 @@ cudaError_t launch_one(rtp_handle* h, int kind, Kernel k, dim3 grid, dim3 block,
 rtp_status enqueue_layer(rtp_handle* h, const LayerArgs& a0, cudaStream_t s) {
   cudaError_t e;
   if (!a0.dense && a0.nret > 0) {
-    e = launch_one(h, 0, select_kernel, dim3(h->select_grid), dim3(kSelThreads), h->select_smem,
-                   s, true, a0, h->ws);
+    // the ranges are at most ceil(B * nret * max_ctx / grid) tokens: on chip when that fits
+    const long long worst = (long long)a0.B * a0.nret * a0.max_ctx;
+    const bool fits = (worst + h->select_grid - 1) / h->select_grid <= kScoreCap;
+    e = launch_one(h, 0, fits ? select_kernel<true> : select_kernel<false>, dim3(h->select_grid),
+                   dim3(kSelThreads), h->select_smem, s, true, a0, h->ws);
     if (e != cudaSuccess) return cuda_fail(e, "select_kernel launch");
   }
-  LayerArgs a = a0;
-  a.heads = kHeadsAll;
+  const LayerArgs& a = a0;
   e = launch_one(h, 1, attend_kernel, dim3(h->attend_grid), dim3(kAttendThreads), h->attend_smem,
                  s, false, a, h->ws);
   if (e != cudaSuccess) return cuda_fail(e, "attend_kernel launch");
   e = launch_one(h, 2, merge_kernel, dim3(merge_units(a.B * a.Hkv, a.G)), dim3(kMergeThreads),
-                 0, s, false, a, h->ws, h->attend_grid);
+                 0, s, false, a, h->ws);
   return e == cudaSuccess ? RTP_OK : cuda_fail(e, "merge_kernel launch");
 }
 
@@ -300,12 +302,19 @@ rtp_status rtp_create(const rtp_config* cfg, int device, rtp_handle** out) {
   if (h->attend_grid > kMaxPieces) h->attend_grid = kMaxPieces;
 
   h->select_smem = select_smem_bytes(cfg->batch * cfg->num_kv_heads);
-  e = cudaFuncSetAttribute(select_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+  e = cudaFuncSetAttribute(select_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            (int)h->select_smem);
-  int sel_per_sm = 0;
   if (e == cudaSuccess)
-    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&sel_per_sm, select_kernel, kSelThreads,
-                                                      h->select_smem);
+    e = cudaFuncSetAttribute(select_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)h->select_smem);
+  int sel_per_sm = 0, sel_per_sm_spill = 0;
+  if (e == cudaSuccess)
+    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&sel_per_sm, select_kernel<true>,
+                                                      kSelThreads, h->select_smem);
+  if (e == cudaSuccess)
+    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&sel_per_sm_spill, select_kernel<false>,
+                                                      kSelThreads, h->select_smem);
+  if (sel_per_sm_spill < sel_per_sm) sel_per_sm = sel_per_sm_spill;  // one grid for both
   if (e != cudaSuccess || sel_per_sm < 1) {
     delete h;
     return e != cudaSuccess ? cuda_fail(e, "occupancy of select_kernel")
@@ -346,11 +355,12 @@ rtp_status rtp_create(const rtp_config* cfg, int device, rtp_handle** out) {
   w.bstar = reinterpret_cast<int*>(base + p.off[4]);
   w.mass_total = reinterpret_cast<unsigned long long*>(base + p.off[5]);
   w.sel_idx = reinterpret_cast<int*>(base + p.off[6]);
-  w.cta_bins = reinterpret_cast<uint32_t*>(base + p.off[7]);
+  w.cta_ge = reinterpret_cast<uint32_t*>(base + p.off[7]);
+  w.bins = reinterpret_cast<unsigned char*>(base + p.off[8]);
   w.sel_total = reinterpret_cast<int*>(base + p.off[9]);
   w.sel_n = reinterpret_cast<int*>(base + p.off[10]);
   w.grid_bar = reinterpret_cast<unsigned*>(base + p.off[11]);
-  w.head_off = reinterpret_cast<long long*>(base + p.off[13]);
+  w.head_pieces = reinterpret_cast<int2*>(base + p.off[13]);
   w.partials = reinterpret_cast<float*>(base + p.off[14]);
   w.status = reinterpret_cast<unsigned*>(base + p.off[15]);
   w.ld = (int)round_up((size_t)cfg->max_ctx, 64);
@@ -537,6 +547,8 @@ rtp_status rtp_get_device_status(rtp_handle* h, uint32_t* code) {
   cudaError_t e = cudaDeviceSynchronize();
   if (e == cudaSuccess) e = cudaMemcpy(code, h->ws.status, 4, cudaMemcpyDeviceToHost);
   if (e == cudaSuccess) e = cudaMemset(h->ws.status, 0, 4);
+  // a barrier that timed out leaves its counter mid-count: start the next launch from zero
+  if (e == cudaSuccess && (*code & kDevWaitTimeout)) e = cudaMemset(h->ws.grid_bar, 0, 4);
   if (e != cudaSuccess) return cuda_fail(e, "reading the device status");
   if (*code) return fail(RTP_ERR_DEVICE_STATUS, "device status 0x%x", *code);
   return ok();

@@ -37,10 +37,34 @@ __device__ __forceinline__ void pdl_launch_dependents() {
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 }
 
+// Atomic add at GPU scope with release (publishes the writes the thread ordered before it) and
+// acquire (later reads see what other releasing threads published) semantics.
+__device__ __forceinline__ unsigned atomic_add_acq_rel_gpu(unsigned* p, unsigned v) {
+  unsigned old;
+  asm volatile("atom.acq_rel.gpu.global.add.u32 %0, [%1], %2;" : "=r"(old) : "l"(p), "r"(v)
+               : "memory");
+  return old;
+}
+
 __device__ __forceinline__ unsigned ld_acquire_gpu(const unsigned* p) {
   unsigned v;
   asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
   return v;
+}
+
+// floor(num / den) for 0 <= num < 2^53 and den >= 1, without a 64-bit integer division: the
+// double quotient is within one of the result, and one integer check each way corrects it.
+__device__ __forceinline__ long long floor_div(long long num, long long den) {
+  long long q = (long long)((double)num / (double)den);
+  if (q * den > num) --q;
+  else if ((q + 1) * den <= num) ++q;
+  return q;
+}
+
+// CTA c whose range [floor(c T / P), floor((c + 1) T / P)) holds position x, for 0 <= x < T,
+// 1 <= P <= T and (x + 1) P + T < 2^53.
+__device__ __forceinline__ long long cta_of(long long x, long long T, long long P) {
+  return floor_div((x + 1) * P + T - 1, T) - 1;
 }
 
 __device__ __forceinline__ unsigned long long global_ns() {

@@ -13,19 +13,20 @@ constexpr int kMaxKvHeads = 256;
 // Device workspace owned by a handle. Slot = b * nret + j for the j-th retrieval KV head of
 // the current layer (the workspace is sized for nret = Hkv).
 struct Workspace {
-  float* scores;                  // [slots][ld]             scaled indexer scores
+  float* scores;                  // [slots][ld]             scaled indexer scores (spill)
+  unsigned char* bins;            // [slots][ld]             their histogram bins (spill)
   float* cta_max;                 // [slots][select_ctas]    per-CTA maxima of the scores
-  unsigned long long* hist;       // [slots][256]            fixed-point (2^-40) bin masses
+  unsigned long long* hist;       // [kHistCopies][slots][256] fixed-point (2^-40) bin masses
   float* s_max;                   // [slots]
   int* bstar;                     // [slots]
   unsigned long long* mass_total; // [slots]                 C_0 in fixed point
   int* sel_idx;                   // [slots][ld]             selected positions, ascending
-  uint32_t* cta_bins;             // [slots][select_ctas][256] tokens per bin, per scoring CTA
+  uint32_t* cta_ge;               // [slots][256][select_ctas] tokens of a CTA in bins >= b
   int* sel_total;                 // [slots]                 |S|
   int* sel_n;                     // [slots]                 N the selection was made over
-  unsigned* grid_bar;             // grid barrier of the selection kernel: generation, root, groups
+  unsigned* grid_bar;             // [0]: grid barrier counter of the selection kernel
   float* partials;                // [(attend_ctas + B*Hkv)][kPartFloats]  piece of CTA c, head h at c + h
-  long long* head_off;            // [B*Hkv + 1]             prefix sums of the heads' token-set sizes
+  int2* head_pieces;              // [B*Hkv]                 first and last attention CTA of a head
   unsigned* status;               // [1] RTP_DEV_* bits
   int ld;                         // per-slot stride of scores / sel_idx: max_ctx rounded up to 64
 };
@@ -41,18 +42,17 @@ struct LayerArgs {
   int* sel_count;                 // [B][Hkv] or nullptr
   int B, Hq, Hkv, G, max_ctx, window, sinks, nret;
   int dense;                      // every head attends over all N tokens
-  int heads;                      // attention launch: kHeadsAll, kHeadsLocal or kHeadsRetrieval
   float top_p, idx_scale, attn_scale_log2, bin_scale;
   short ret_kvh[kMaxKvHeads];     // KV head of retrieval index j (j < nret)
   short slot_of_kvh[kMaxKvHeads]; // retrieval index j of KV head kvh, or -1 for a local head
 };
 
-enum : int { kHeadsAll = 0, kHeadsLocal = 1, kHeadsRetrieval = 2 };
-
 // Kernel entry points (defined in select_kernels.cu / attend_kernel.cu).
-__global__ void select_kernel(const LayerArgs a, const Workspace w);  // cooperative launch
+// cooperative launch; kFits: every CTA's range fits in shared memory (no spill code)
+template <bool kFits>
+__global__ void select_kernel(const LayerArgs a, const Workspace w);
 __global__ void attend_kernel(const LayerArgs a, const Workspace w);
-__global__ void merge_kernel(const LayerArgs a, const Workspace w, int attend_grid);
+__global__ void merge_kernel(const LayerArgs a, const Workspace w);
 
 constexpr int kAttendWarps = 4;                          // warps per attention CTA
 constexpr int kAttendDepth = 3;                          // cp.async stages per warp
@@ -63,6 +63,7 @@ constexpr int kMaxAttendHeads = 1024;                    // B * Hkv per layer
 constexpr int kMaxSelSlots = kMaxAttendHeads;            // retrieval slots per layer
 constexpr int kMaxSelectCtasPerSm = 2;                   // resident selection CTAs per SM
 constexpr int kScoreCap = 16384;                         // scores a selection CTA keeps on chip
+constexpr int kHistCopies = 8;                           // copies of each slot's histogram
 size_t select_smem_bytes(int slots);
 constexpr int kMaxPieces = 1024;                         // attention CTAs (pieces of one head)
 constexpr int kMergeThreads = 128;

@@ -9,17 +9,19 @@
 // One persistent cooperative launch per layer selects the tokens of every retrieval slot
 // (slot = b * nret + j for the j-th retrieval KV head). The indexer keys of all slots are laid
 // end to end and cut into one equal range per CTA; a CTA keeps the scores of its range in its
-// own shared memory (ranges longer than kScoreCap spill the rest to a global buffer). Three
-// phases, two grid barriers (bounded waits):
+// own shared memory (ranges longer than kScoreCap spill the rest to global buffers; the host
+// launches the variant without spill code when no range can be that long). Three phases, two
+// grid barriers (bounded waits):
 //   1. scores: a lane pair reads a token's 32 bytes with two 16-byte loads (double-buffered),
 //      the scaled fp32 score is kept, and each CTA records the max of each slot it scores;
 //   2. histogram: s_max of a slot = max of its CTAs' maxima; every score is binned relative
 //      to s_max and exp(s - s_max) is added in 2^-40 fixed point to per-warp shared bins
-//      (32-bit words, exact integer sums whatever the order). The CTA adds its masses to the
-//      slot's global histogram (integer atomics) and stores its token count per bin;
-//   3. compaction: each CTA computes b* from the slot's histogram (one warp, suffix sums from
-//      the top bin), its offset from the bin counts (bins >= b*) of the CTAs before it, and
-//      writes its selected positions, ascending, into one dense list per slot.
+//      (32-bit words, exact integer sums whatever the order). The CTA adds its masses to one
+//      of kHistCopies copies of the slot's global histogram (integer atomics, spread over the
+//      copies) and stores, per bin b, how many of its tokens fall in bins >= b;
+//   3. compaction: each CTA sums the copies, finds b* with a CTA-wide suffix scan over the
+//      bins, reads the counts at b* of the CTAs before it (one coalesced load) for its offset,
+//      and writes its selected positions, ascending, into one dense list per slot.
 // Phases 2 and 3 bin the same fp32 scores with score_bin, so counts and flags agree exactly.
 #include "rtp_device.cuh"
 #include "rtp_kernels.h"
@@ -29,11 +31,11 @@ namespace rtp {
 namespace {
 
 constexpr int kWarpsSel = kSelThreads / 32;
-constexpr int kRowUnroll = 16;  // independent 16-byte loads per thread in the offset sums
+static_assert(kSelThreads == kBins, "phase 3 gives one bin to each thread");
 
 __device__ __forceinline__ int clamp_seq_len(const LayerArgs& a, int b, unsigned* status,
                                              bool report) {
-  int n = a.seq_lens[b];
+  int n = __ldcg(a.seq_lens + b);
   if (n < 1 || n > a.max_ctx) {
     if (report) atomicOr(status, kDevBadSeqlen);
     n = n < 1 ? 1 : a.max_ctx;
@@ -90,102 +92,56 @@ __device__ __forceinline__ int block_excl_scan(int v, int& excl, int* red) {
   return all;
 }
 
-// Grid-wide barrier of a cooperative launch (every CTA is resident). Arrivals go through one
-// counter per group of kBarGroup CTAs, then the group's last arrival through the root counter;
-// the root's last arrival bumps the generation word. The wait gives up after kWaitLimitNs, sets
-// kDevWaitTimeout and makes later barriers of the CTA return at once, so the kernel ends.
-// bar: [0] generation, [1] root counter, [2 ..] group counters.
-constexpr int kBarGroup = 16;
+// Inclusive suffix sum over the CTA's threads (thread i gets the sum of threads >= i).
+template <typename T>
+__device__ __forceinline__ T block_suffix_sum(T v, T* red) {
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  T x = v;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const T y = __shfl_down_sync(0xffffffffu, x, o);
+    if (lane + o < 32) x += y;
+  }
+  __syncthreads();
+  if (lane == 0) red[warp] = x;
+  __syncthreads();
+  T after = 0;
+#pragma unroll
+  for (int k = 0; k < kWarpsSel; ++k) after += (k > warp) ? red[k] : (T)0;
+  return x + after;
+}
+
+// Grid-wide barrier of a cooperative launch (every CTA is resident), one counter whose top bit
+// flips once per barrier: CTA 0 adds 2^31 - (P - 1), every other CTA adds 1, so the low 31
+// bits (0 between barriers) reach 2^31 and carry into the top bit exactly at the last arrival.
+// The add has release semantics (it publishes the CTA's writes) and the polling load acquire
+// semantics. The wait gives up after kWaitLimitNs, sets kDevWaitTimeout and makes later
+// barriers of the CTA return at once, so the kernel ends (the host then clears the counter).
 __device__ void grid_barrier(unsigned* bar, unsigned* status, int* aborted) {
   __syncthreads();
   if (threadIdx.x == 0 && !*aborted) {
-    const unsigned gen = ld_acquire_gpu(bar);
-    __threadfence();
-    const unsigned grp = blockIdx.x / kBarGroup;
-    const unsigned ngrp = (gridDim.x + kBarGroup - 1) / kBarGroup;
-    const unsigned in_grp = min((unsigned)kBarGroup, gridDim.x - grp * kBarGroup);
-    bool released = false;
-    if (atomicAdd(bar + 2 + grp, 1u) == in_grp - 1u) {
-      atomicExch(bar + 2 + grp, 0u);
-      if (atomicAdd(bar + 1, 1u) == ngrp - 1u) {
-        atomicExch(bar + 1, 0u);
-        __threadfence();
-        atomicAdd(bar, 1u);
-        released = true;
+    const unsigned inc = (blockIdx.x == 0) ? 0x80000000u - (gridDim.x - 1u) : 1u;
+    const unsigned old = atomic_add_acq_rel_gpu(bar, inc);
+    const unsigned long long t0 = global_ns();
+    unsigned it = 0;
+    while (((ld_acquire_gpu(bar) ^ old) & 0x80000000u) == 0u) {
+      if ((++it & 255u) == 0 && global_ns() - t0 > kWaitLimitNs) {
+        atomicOr(status, kDevWaitTimeout);
+        *aborted = 1;
+        break;
       }
     }
-    if (!released) {
-      const unsigned long long t0 = global_ns();
-      unsigned it = 0;
-      while (ld_acquire_gpu(bar) == gen) {
-        if ((++it & 255u) == 0 && global_ns() - t0 > kWaitLimitNs) {
-          atomicOr(status, kDevWaitTimeout);
-          *aborted = 1;
-          break;
-        }
-      }
-    }
-    __threadfence();
   }
   __syncthreads();
 }
 
-// Largest s < S with off[s] <= x (off ascending, off[0] = 0 <= x < off[S]).
-__device__ __forceinline__ int upper_slot(const long long* off, int S, long long x) {
-  int lo = 0, hi = S - 1;
-  while (lo < hi) {
-    const int mid = (lo + hi + 1) >> 1;
-    if (off[mid] <= x) lo = mid; else hi = mid - 1;
-  }
-  return lo;
-}
-
-// CTA whose range [floor(c T / P), floor((c+1) T / P)) holds position x (0 <= x < T, P <= T).
-__device__ __forceinline__ long long cta_of(long long x, long long T, long long P) {
-  return ((x + 1) * P + T - 1) / T - 1;
-}
-
-// The scores of this CTA's range: the first kScoreCap in shared memory, the rest (if any) in
-// the global buffer at their slot positions.
-struct Scores {
-  float* sm;        // shared, indexed by position in the CTA range
-  float* glob;      // global scores workspace
-  size_t ld;
-  long long t0;     // range start (concatenated coordinates)
-  const long long* soff;
-  __device__ float* at(int s, int n) const {
-    const long long i = soff[s] + n - t0;
-    return (i < kScoreCap) ? sm + i : glob + (size_t)s * ld + n;
-  }
-};
-
-}  // namespace
-
-size_t select_smem_bytes(int slots) {
-  return (size_t)kScoreCap * 4 + (size_t)(slots + 1) * 8;
-}
-
-__global__ void __launch_bounds__(kSelThreads, 2) select_kernel(const LayerArgs a, const Workspace w) {
-  extern __shared__ __align__(16) unsigned char dsm[];
-  __shared__ uint32_t wlo[kWarpsSel][kBins];   // per-warp fixed-point masses, low words
-  __shared__ uint32_t whi[kWarpsSel][kBins];   // high words
-  __shared__ uint32_t cnt[kBins];              // tokens per bin in the segment
-  __shared__ float redf[kWarpsSel];
-  __shared__ int redi[kWarpsSel];
-  __shared__ int aborted;
-  __shared__ int bstar_s;
-
+// Slot sizes (clamped sequence lengths) and their prefix sums into soff[0 .. S]. report: flag
+// out-of-range lengths in the status word.
+__device__ void slot_offsets(const LayerArgs& a, int S, long long* soff, unsigned* status,
+                             bool report) {
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int S = a.B * a.nret;
-  float* s_scores = reinterpret_cast<float*>(dsm);
-  long long* soff = reinterpret_cast<long long*>(dsm + (size_t)kScoreCap * 4);
-  if (tid == 0) aborted = 0;
-  pdl_wait();
-  pdl_launch_dependents();
-
-  // slot sizes and their prefix sums
   for (int s = tid; s < S; s += kSelThreads)
-    soff[s + 1] = clamp_seq_len(a, s / a.nret, w.status, blockIdx.x == 0 && (s % a.nret) == 0);
+    soff[s + 1] = clamp_seq_len(a, s / a.nret, status, report && (s % a.nret) == 0);
   __syncthreads();
   if (warp == 0) {  // inclusive scan, 32 slots at a time
     long long carry = 0;
@@ -202,16 +158,82 @@ __global__ void __launch_bounds__(kSelThreads, 2) select_kernel(const LayerArgs 
     }
     if (lane == 0) soff[0] = 0;
   }
-  if (blockIdx.x == 0)  // phase 2 accumulates into these
-    for (int i = tid; i < S * kBins; i += kSelThreads) w.hist[i] = 0ull;
   __syncthreads();
+}
+
+// Largest s < S with off[s] <= x (off ascending, off[0] = 0 <= x < off[S]).
+__device__ __forceinline__ int upper_slot(const long long* off, int S, long long x) {
+  int lo = 0, hi = S - 1;
+  while (lo < hi) {
+    const int mid = (lo + hi + 1) >> 1;
+    if (off[mid] <= x) lo = mid; else hi = mid - 1;
+  }
+  return lo;
+}
+
+// The scores (fp32) and bins (one byte) of this CTA's range: the first kScoreCap of each in
+// shared memory, the rest (if any) in the global spill buffers at their slot positions. When
+// the whole range fits (the usual case) the loops index shared memory directly.
+template <bool kFits>
+struct Scores {
+  float* sm;              // shared, indexed by position in the CTA range
+  unsigned char* smb;
+  float* glob;            // global spill buffers
+  unsigned char* globb;
+  size_t ld;
+  long long t0;           // range start (concatenated coordinates)
+  const long long* soff;
+  __device__ float* at(int s, int n) const {
+    const long long i = soff[s] + n - t0;
+    if (kFits) return sm + i;
+    return (i < kScoreCap) ? sm + i : glob + (size_t)s * ld + n;
+  }
+  __device__ unsigned char* bin_at(int s, int n) const {
+    const long long i = soff[s] + n - t0;
+    if (kFits) return smb + i;
+    return (i < kScoreCap) ? smb + i : globb + (size_t)s * ld + n;
+  }
+};
+
+}  // namespace
+
+size_t select_smem_bytes(int slots) {
+  return (size_t)kScoreCap * 5 + (size_t)(slots + 1) * 8;
+}
+
+template <bool kFits>
+__global__ void __launch_bounds__(kSelThreads, 2) select_kernel(const LayerArgs a, const Workspace w) {
+  extern __shared__ __align__(16) unsigned char dsm[];
+  __shared__ uint32_t wlo[kWarpsSel][kBins];   // per-warp fixed-point masses, bits 0..19
+  __shared__ uint32_t whi[kWarpsSel][kBins];   // bits 20..40
+  __shared__ uint32_t cnt[kBins];              // tokens per bin in the segment
+  __shared__ float redf[kWarpsSel];
+  __shared__ int redi[kWarpsSel];
+  __shared__ int aborted;
+  __shared__ int bstar_s;
+
+  __shared__ unsigned long long red64[kWarpsSel];
+
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int S = a.B * a.nret;
+  float* s_scores = reinterpret_cast<float*>(dsm);
+  unsigned char* s_bins = dsm + (size_t)kScoreCap * 4;
+  long long* soff = reinterpret_cast<long long*>(dsm + (size_t)kScoreCap * 5);
+  if (tid == 0) aborted = 0;
+
+  pdl_wait();
+  pdl_launch_dependents();
+
+  slot_offsets(a, S, soff, w.status, blockIdx.x == 0);
+  if (blockIdx.x == 0)  // phase 2 accumulates into these
+    for (int i = tid; i < kHistCopies * S * kBins; i += kSelThreads) w.hist[i] = 0ull;
 
   const long long T = soff[S];
   const long long P = min((long long)gridDim.x, T);
   const bool active = (long long)blockIdx.x < P;
-  const long long t0 = active ? (long long)blockIdx.x * T / P : 0;
-  const long long t1 = active ? ((long long)blockIdx.x + 1) * T / P : 0;
-  const Scores sc{s_scores, w.scores, (size_t)w.ld, t0, soff};
+  const long long t0 = active ? floor_div((long long)blockIdx.x * T, P) : 0;
+  const long long t1 = active ? floor_div(((long long)blockIdx.x + 1) * T, P) : 0;
+  const Scores<kFits> sc{s_scores, s_bins, w.scores, w.bins, (size_t)w.ld, t0, soff};
 
   // ---- phase 1: indexer scores of this CTA's range -----------------------------------------
   if (active) {
@@ -297,27 +319,40 @@ __global__ void __launch_bounds__(kSelThreads, 2) select_kernel(const LayerArgs 
       }
       cnt[tid] = 0u;
       const float s_max = block_max(m, redf);  // its barriers also order the zero fill
-      for (int n = n0 + tid; n < n1; n += kSelThreads) {
-        const float v = *sc.at(s, n);
-        const int bin = score_bin(v, s_max, a.bin_scale);
-        const float wgt = expf(v - s_max);                          // in (0, 1]
-        const unsigned long long fx = __float2ull_rn(wgt * 1099511627776.0f);  // * 2^40, exact
-        const uint32_t lo = (uint32_t)fx;
-        uint32_t hi = (uint32_t)(fx >> 32);
-        if (lo) {
-          const uint32_t old = atomicAdd(&wlo[warp][bin], lo);
-          hi += (old + lo < old) ? 1u : 0u;                          // carry out of the low word
+      const int copy = (int)(blockIdx.x % kHistCopies);
+      // bits 0..19 and 20..40 of the 2^-40 weights go to separate 32-bit words, so that no add
+      // needs the old value: a warp adds at most kScoreCap / 8 tokens to a bin before the flush
+      for (int k0 = n0; k0 < n1; k0 += kScoreCap) {
+        const int k1 = min(n1, k0 + kScoreCap);
+        if (k0 != n0) {
+          for (int i = tid; i < kWarpsSel * kBins; i += kSelThreads) {
+            (&wlo[0][0])[i] = 0u;
+            (&whi[0][0])[i] = 0u;
+          }
+          __syncthreads();
         }
-        if (hi) atomicAdd(&whi[warp][bin], hi);
-        atomicAdd(&cnt[bin], 1u);
-      }
-      __syncthreads();
-      unsigned long long v = 0ull;
+#pragma unroll 4
+        for (int n = k0 + tid; n < k1; n += kSelThreads) {
+          const float v = *sc.at(s, n);
+          const int bin = score_bin(v, s_max, a.bin_scale);
+          *sc.bin_at(s, n) = (unsigned char)bin;
+          const float wgt = expf(v - s_max);                          // in (0, 1]
+          const unsigned long long fx = __float2ull_rn(wgt * 1099511627776.0f);  // * 2^40, exact
+          atomicAdd(&wlo[warp][bin], (uint32_t)fx & 0xFFFFFu);
+          atomicAdd(&whi[warp][bin], (uint32_t)(fx >> 20));
+          atomicAdd(&cnt[bin], 1u);
+        }
+        __syncthreads();
+        unsigned long long v = 0ull;
 #pragma unroll
-      for (int k = 0; k < kWarpsSel; ++k)
-        v += ((unsigned long long)whi[k][tid] << 32) + wlo[k][tid];
-      if (v) atomicAdd(w.hist + (size_t)s * kBins + tid, v);
-      w.cta_bins[((size_t)s * gridDim.x + blockIdx.x) * kBins + tid] = cnt[tid];
+        for (int k = 0; k < kWarpsSel; ++k)
+          v += ((unsigned long long)whi[k][tid] << 20) + wlo[k][tid];
+        if (v) atomicAdd(w.hist + ((size_t)copy * S + s) * kBins + tid, v);
+        __syncthreads();  // the per-warp words are read before the next chunk clears them
+      }
+      // tokens of this CTA in bins >= tid, stored bin-major so that phase 3 reads one column
+      const unsigned ge = block_suffix_sum<unsigned>(cnt[tid], reinterpret_cast<unsigned*>(redi));
+      w.cta_ge[((size_t)s * kBins + tid) * gridDim.x + blockIdx.x] = ge;
       if (blockIdx.x == c0 && tid == 0) w.s_max[s] = s_max;
       __syncthreads();
     }
@@ -333,65 +368,30 @@ __global__ void __launch_bounds__(kSelThreads, 2) select_kernel(const LayerArgs 
       t = soff[s] + n1;
       const int c0 = (int)cta_of(soff[s], T, P), c1 = (int)cta_of(soff[s + 1] - 1, T, P);
       const bool first = (int)blockIdx.x == c0;
-      if (warp == 0) {  // b*: one warp, 8 bins per lane, suffix sums from the top bin down
-        unsigned long long hv[8], lane_sum = 0ull;
+      // b*: thread tid owns bin tid; the copies are summed, then a suffix scan from the top
+      // bin gives each bin's mass at or above it
+      unsigned long long hv = 0ull;
 #pragma unroll
-        for (int i = 0; i < 8; ++i) {
-          hv[i] = __ldcg(w.hist + (size_t)s * kBins + lane * 8 + i);
-          lane_sum += hv[i];
-        }
-        unsigned long long incl = lane_sum;  // sum over lanes >= lane
-#pragma unroll
-        for (int o = 1; o < 32; o <<= 1) {
-          const unsigned long long y = __shfl_down_sync(0xffffffffu, incl, o);
-          if (lane + o < 32) incl += y;
-        }
-        const unsigned long long total = __shfl_sync(0xffffffffu, incl, 0);
-        const double target = (double)a.top_p * (double)total;
-        unsigned long long c = incl - lane_sum;  // mass of the bins above this lane's
-        int best = -1;
-#pragma unroll
-        for (int i = 7; i >= 0; --i) {
-          c += hv[i];
-          if (best < 0 && (double)c >= target) best = lane * 8 + i;
-        }
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) best = max(best, __shfl_xor_sync(0xffffffffu, best, o));
-        if (lane == 0) {
-          bstar_s = best < 0 ? 0 : best;
-          if (first) w.mass_total[s] = total;
-        }
-      }
+      for (int k = 0; k < kHistCopies; ++k)
+        hv += __ldcg(w.hist + ((size_t)k * S + s) * kBins + tid);
+      const unsigned long long sfx = block_suffix_sum<unsigned long long>(hv, red64);
+      __syncthreads();
+      if (tid == 0) red64[0] = sfx;  // the total C_0
+      if (tid == 0) bstar_s = 0;
+      __syncthreads();
+      const unsigned long long total = red64[0];
+      const double target = (double)a.top_p * (double)total;
+      const unsigned long long above = sfx - hv;  // mass of the bins above tid
+      if ((double)sfx >= target && (tid == kBins - 1 || !((double)above >= target)))
+        bstar_s = tid;  // the highest bin whose suffix mass reaches p * C_0 (one thread)
       __syncthreads();
       const int bs = bstar_s;
-      // selected tokens of the slot's CTAs before this one (first CTA: of all, for |S|); the
-      // (CTA, 4-bin group) pairs are spread over the threads so their 16-byte loads overlap
+      if (first && tid == 0) w.mass_total[s] = total;
+      // selected tokens of the slot's CTAs before this one (first CTA: of all, for |S|)
       const int r0 = c0, r1 = first ? c1 + 1 : (int)blockIdx.x;
-      const int b4 = bs & ~3, ngrp = (kBins - b4) >> 2;
-      const uint32_t* rows_base = w.cta_bins + (size_t)s * gridDim.x * kBins + b4;
-      const int E = (r1 - r0) * ngrp;
+      const unsigned* col = w.cta_ge + ((size_t)s * kBins + bs) * gridDim.x;
       int mine = 0;
-      for (int e0 = 0; e0 < E; e0 += kSelThreads * kRowUnroll) {
-        uint4 q4[kRowUnroll];
-#pragma unroll
-        for (int k = 0; k < kRowUnroll; ++k) {
-          const int e = e0 + k * kSelThreads + tid;
-          q4[k] = (e < E) ? __ldcg(reinterpret_cast<const uint4*>(
-                                rows_base + (size_t)(r0 + e / ngrp) * kBins + (e % ngrp) * 4))
-                          : make_uint4(0, 0, 0, 0);
-        }
-#pragma unroll
-        for (int k = 0; k < kRowUnroll; ++k) {
-          const int e = e0 + k * kSelThreads + tid;
-          if ((e % ngrp) == 0) {  // first group of a row: drop the bins below b*
-            const int lo = bs - b4;
-            q4[k].x = (lo > 0) ? 0u : q4[k].x;
-            q4[k].y = (lo > 1) ? 0u : q4[k].y;
-            q4[k].z = (lo > 2) ? 0u : q4[k].z;
-          }
-          mine += (int)(q4[k].x + q4[k].y + q4[k].z + q4[k].w);
-        }
-      }
+      for (int c = r0 + tid; c < r1; c += kSelThreads) mine += (int)__ldcg(col + c);
       const int sum_rows = block_sum(mine, redi);
       int base = first ? 0 : sum_rows;
       if (first && tid == 0) {
@@ -399,7 +399,6 @@ __global__ void __launch_bounds__(kSelThreads, 2) select_kernel(const LayerArgs 
         w.sel_total[s] = sum_rows;
         w.sel_n[s] = (int)(soff[s + 1] - soff[s]);
       }
-      const float s_max = __ldcg(w.s_max + s);
       int* out = w.sel_idx + (size_t)s * w.ld;
       // ordered compaction: warp w takes 32 x kPerThread consecutive tokens of each round, one
       // ballot per 32; the warps' counts are scanned, then each warp writes its tokens in order
@@ -411,7 +410,8 @@ __global__ void __launch_bounds__(kSelThreads, 2) select_kernel(const LayerArgs 
 #pragma unroll
         for (int k = 0; k < kPerThread; ++k) {
           const int n = wb + 32 * k + lane;
-          const bool f = n < n1 && score_bin(*sc.at(s, n), s_max, a.bin_scale) >= bs;
+          const int bin = *sc.bin_at(s, min(n, n1 - 1));  // in range: no branch around the load
+          const bool f = n < n1 && bin >= bs;
           bal[k] = __ballot_sync(0xffffffffu, f);
           wcnt += __popc(bal[k]);
         }
@@ -430,5 +430,8 @@ __global__ void __launch_bounds__(kSelThreads, 2) select_kernel(const LayerArgs 
     }
   }
 }
+
+template __global__ void select_kernel<true>(const LayerArgs, const Workspace);
+template __global__ void select_kernel<false>(const LayerArgs, const Workspace);
 
 }  // namespace rtp

@@ -171,7 +171,9 @@ RTP_API rtp_status rtp_profile_enable(rtp_handle *h, int enable);
 RTP_API rtp_status rtp_profile_read(rtp_handle *h, double *ms, int64_t *launches);
 
 /* Reads and clears the device status word (RTP_DEV_* bits) after synchronising the device.
- * Returns RTP_ERR_DEVICE_STATUS when a bit was set, RTP_OK otherwise. */
+ * After RTP_DEV_WAIT_TIMEOUT it also resets the selection kernel's grid-barrier counter, so
+ * that later calls on the handle start from a clean barrier. Returns RTP_ERR_DEVICE_STATUS
+ * when a bit was set, RTP_OK otherwise. */
 RTP_API rtp_status rtp_get_device_status(rtp_handle *h, uint32_t *code);
 
 /* ---- Attention without any allocation --------------------------------------------------

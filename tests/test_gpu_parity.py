@@ -106,6 +106,21 @@ def test_all_retrieval_heads():
     _run(p)
 
 
+@pytest.mark.slow
+def test_selection_ranges_beyond_on_chip_capacity():
+    """Eight retrieval slots of 655 360 tokens: each selection CTA scores more tokens than it
+    keeps in shared memory, so part of its scores and bins go through the global spill
+    buffers, and its histogram is flushed in more than one chunk."""
+    N = 655360
+    kinds = [[W.KIND_CONC, W.KIND_DIFFUSE, W.KIND_FLAT, W.KIND_CONC],
+             [W.KIND_DIFFUSE, W.KIND_CONC, W.KIND_CONC, W.KIND_FLAT]]
+    p = W.custom(batch=2, num_q_heads=32, num_kv_heads=4, seq_lens=[N, N - 4321], max_ctx=N,
+                 retrieval=[1, 1, 1, 1], kinds=kinds, n_needles=[[2, 0, 0, 7], [0, 5, 3, 0]],
+                 seed=21)
+    assert sum(p.seq_lens) * 4 > 148 * 2 * 16384  # more than the CTAs keep on chip
+    _run(p, exact=False)
+
+
 def test_dense_decode_matches_oracle():
     p = W.custom(batch=2, num_q_heads=32, num_kv_heads=4, seq_lens=[33000, 7],
                  max_ctx=33000, retrieval=[1, 0, 0, 0],
