@@ -221,7 +221,7 @@ rtp_status enqueue_layer(rtp_handle* h, const LayerArgs& a0, cudaStream_t s) {
     // the ranges are at most ceil(B * nret * max_ctx / grid) tokens: on chip when that fits
     const long long worst = (long long)a0.B * a0.nret * a0.max_ctx;
     const bool fits = (worst + h->select_grid - 1) / h->select_grid <= kScoreCap;
-    e = launch_one(h, 0, fits ? select_kernel<true> : select_kernel<false>, dim3(h->select_grid),
+    e = launch_one(h, 0, fits ? select_kernel_onchip : select_kernel_spill, dim3(h->select_grid),
                    dim3(kSelThreads), h->select_smem, s, true, a0, h->ws);
     if (e != cudaSuccess) return cuda_fail(e, "select_kernel launch");
   }
@@ -302,17 +302,17 @@ rtp_status rtp_create(const rtp_config* cfg, int device, rtp_handle** out) {
   if (h->attend_grid > kMaxPieces) h->attend_grid = kMaxPieces;
 
   h->select_smem = select_smem_bytes(cfg->batch * cfg->num_kv_heads);
-  e = cudaFuncSetAttribute(select_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+  e = cudaFuncSetAttribute(select_kernel_onchip, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            (int)h->select_smem);
   if (e == cudaSuccess)
-    e = cudaFuncSetAttribute(select_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    e = cudaFuncSetAttribute(select_kernel_spill, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              (int)h->select_smem);
   int sel_per_sm = 0, sel_per_sm_spill = 0;
   if (e == cudaSuccess)
-    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&sel_per_sm, select_kernel<true>,
+    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&sel_per_sm, select_kernel_onchip,
                                                       kSelThreads, h->select_smem);
   if (e == cudaSuccess)
-    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&sel_per_sm_spill, select_kernel<false>,
+    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&sel_per_sm_spill, select_kernel_spill,
                                                       kSelThreads, h->select_smem);
   if (sel_per_sm_spill < sel_per_sm) sel_per_sm = sel_per_sm_spill;  // one grid for both
   if (e != cudaSuccess || sel_per_sm < 1) {

@@ -48,9 +48,10 @@ struct LayerArgs {
 };
 
 // Kernel entry points (defined in select_kernels.cu / attend_kernel.cu).
-// cooperative launch; kFits: every CTA's range fits in shared memory (no spill code)
-template <bool kFits>
-__global__ void select_kernel(const LayerArgs a, const Workspace w);
+// Cooperative launches. _onchip: every CTA's range fits in shared memory (no spill code);
+// _spill: longer ranges keep the rest of their scores and bins in the global workspace.
+__global__ void select_kernel_onchip(const LayerArgs a, const Workspace w);
+__global__ void select_kernel_spill(const LayerArgs a, const Workspace w);
 __global__ void attend_kernel(const LayerArgs a, const Workspace w);
 __global__ void merge_kernel(const LayerArgs a, const Workspace w);
 

@@ -202,7 +202,7 @@ size_t select_smem_bytes(int slots) {
 }
 
 template <bool kFits>
-__global__ void __launch_bounds__(kSelThreads, 2) select_kernel(const LayerArgs a, const Workspace w) {
+__device__ __forceinline__ void select_body(const LayerArgs& a, const Workspace& w) {
   extern __shared__ __align__(16) unsigned char dsm[];
   __shared__ uint32_t wlo[kWarpsSel][kBins];   // per-warp fixed-point masses, bits 0..19
   __shared__ uint32_t whi[kWarpsSel][kBins];   // bits 20..40
@@ -431,7 +431,14 @@ __global__ void __launch_bounds__(kSelThreads, 2) select_kernel(const LayerArgs 
   }
 }
 
-template __global__ void select_kernel<true>(const LayerArgs, const Workspace);
-template __global__ void select_kernel<false>(const LayerArgs, const Workspace);
+__global__ void __launch_bounds__(kSelThreads, 2) select_kernel_onchip(const LayerArgs a,
+                                                                       const Workspace w) {
+  select_body<true>(a, w);
+}
+
+__global__ void __launch_bounds__(kSelThreads, 2) select_kernel_spill(const LayerArgs a,
+                                                                      const Workspace w) {
+  select_body<false>(a, w);
+}
 
 }  // namespace rtp
