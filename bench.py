@@ -178,6 +178,44 @@ def oracle_sample(plan, layer_fn, layers, threads):
     return secs, nbytes
 
 
+def dist_env() -> tuple[int, int, int]:
+    """(world, rank, local rank) as torchrun sets them; (1, 0, 0) without torchrun."""
+    return (int(os.environ.get("WORLD_SIZE", "1")), int(os.environ.get("RANK", "0")),
+            int(os.environ.get("LOCAL_RANK", "0")))
+
+
+def init_dist(local: int):
+    """One process per GPU over NCCL (gloo when no GPU is visible, for the host-side tests),
+    with a short timeout so that ranks waiting on a dead peer end with an error."""
+    import datetime
+    import torch
+    import torch.distributed as dist
+    if torch.cuda.is_available():
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=600),
+                                device_id=torch.device("cuda", local))
+    else:
+        dist.init_process_group("gloo", timeout=datetime.timedelta(seconds=120))
+
+
+def max_over_ranks(x: float, world: int, device) -> float:
+    """The maximum of x over all ranks (x itself on one rank): a multi-GPU step takes as long as
+    its slowest replica."""
+    if world == 1:
+        return float(x)
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([float(x)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def throughput(world: int, ms_per_step: float) -> float:
+    """Whole-job decode steps per second: every rank decodes its own step (replicas), so the
+    job finishes world steps per max-over-ranks step time."""
+    return world * 1e3 / ms_per_step
+
+
 def run_reference(args, plan, rank, world):
     """--impl reference: the fp64 CPU oracle on the host cores, each step a bounded sample of
     the same workload (one sampled layer), its time scaled to a full step by bytes."""
@@ -242,14 +280,9 @@ def main():
     from head_wise_sparse_retrieval_b200 import rtp
     from head_wise_sparse_retrieval_b200 import workloads as W
 
-    world = int(os.environ.get("WORLD_SIZE", "1"))
-    rank = int(os.environ.get("RANK", "0"))
-    local = int(os.environ.get("LOCAL_RANK", "0"))
+    world, rank, local = dist_env()
     if world > 1:
-        torch.cuda.set_device(local)
-        import datetime
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=600),
-                                device_id=torch.device("cuda", local))
+        init_dist(local)
 
     plan = W.plan(args.workload, top_p=args.top_p, num_layers=args.layers, ctx=args.ctx)
 
@@ -338,11 +371,7 @@ def main():
     if world > 1:
         dist.barrier()
     clocks = sampler.stop() if rank == 0 else {}
-    ms = e0.elapsed_time(e1) / args.steps
-    if world > 1:
-        t = torch.tensor([ms], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms = float(t.item())
+    ms = max_over_ranks(e0.elapsed_time(e1) / args.steps, world, dev)
     del g
 
     # per-kernel durations (CUDA events around each launch on the launch stream)
@@ -414,12 +443,8 @@ def main():
             h.decode_step_host(q_h, qi_h, seq_h, views, masks, plan.top_p, out_h, stream=stream)
         x1.record(stream)
         torch.cuda.synchronize()
-        xms = x0.elapsed_time(x1) / ne
-        if world > 1:
-            t = torch.tensor([xms], device=dev)
-            dist.all_reduce(t, op=dist.ReduceOp.MAX)
-            xms = float(t.item())
-        e2e = {"value": world * 1e3 / xms, "unit": "steps/s",
+        xms = max_over_ranks(x0.elapsed_time(x1) / ne, world, dev)
+        e2e = {"value": throughput(world, xms), "unit": "steps/s",
                "h2d_bytes_per_step": int(q_h.numel() * 2 + qi_h.numel() * 2 + seq_h.numel() * 4),
                "d2h_bytes_per_step": int(out_h.numel() * 4), "ms_per_step": xms}
 
@@ -440,7 +465,7 @@ def main():
                           f"full step by algorithmic bytes"),
                "host_threads": threads}
 
-    value = world * 1e3 / ms
+    value = throughput(world, ms)
     eff_gbs = total_bytes / (ms * 1e-3) / 1e9
     n_sel = [int(s[b, k]) for l, s in enumerate(sel) for b in range(B) for k in range(Hkv)
              if plan.retrieval[l, k]]

@@ -446,7 +446,6 @@ __global__ void __launch_bounds__(kAttendThreads, kAttendCtasPerSm) attend_kerne
     // it ends at the head's size; one piece covering both is the whole head
     const int len = (int)(sOff[hd + 1] - sOff[hd]);
     const bool first_piece = (r0 == 0), last_piece = (r1 == len);
-    const int d = tid;  // 0..127: one output dimension per thread
     float* out_h = a.out + ((size_t)b * a.Hq + (size_t)kvh * a.G) * kHeadDim;
     const bool single = first_piece && last_piece;
     float* piece = w.partials + ((size_t)blockIdx.x + hd) * kPartFloats;
@@ -460,14 +459,16 @@ __global__ void __launch_bounds__(kAttendThreads, kAttendCtasPerSm) attend_kerne
         const float mw = sML[(wq * kMaxGroup + jq) * 2];
         if (mw != -INFINITY) L += sML[(wq * kMaxGroup + jq) * 2 + 1] * exp2f(mw - M);
       }
-      const float O = sO[jq * kOPitch + d];
-      if (single) {
-        out_h[(size_t)jq * kHeadDim + d] = O / L;
-      } else {
-        piece[jq * kHeadDim + d] = O;
-        if (d == 0) {
-          piece[kPartO + jq] = M;
-          piece[kPartO + kMaxGroup + jq] = L;
+      for (int d = tid; d < kHeadDim; d += kAttendThreads) {  // one output dimension per thread
+        const float O = sO[jq * kOPitch + d];
+        if (single) {
+          out_h[(size_t)jq * kHeadDim + d] = O / L;
+        } else {
+          piece[jq * kHeadDim + d] = O;
+          if (d == 0) {
+            piece[kPartO + jq] = M;
+            piece[kPartO + kMaxGroup + jq] = L;
+          }
         }
       }
     }

@@ -55,8 +55,14 @@ __global__ void select_kernel_spill(const LayerArgs a, const Workspace w);
 __global__ void attend_kernel(const LayerArgs a, const Workspace w);
 __global__ void merge_kernel(const LayerArgs a, const Workspace w);
 
-constexpr int kAttendWarps = 4;                          // warps per attention CTA
-constexpr int kAttendDepth = 3;                          // cp.async stages per warp
+#ifndef RTP_ATTEND_WARPS
+#define RTP_ATTEND_WARPS 4
+#endif
+#ifndef RTP_ATTEND_DEPTH
+#define RTP_ATTEND_DEPTH 3
+#endif
+constexpr int kAttendWarps = RTP_ATTEND_WARPS;           // warps per attention CTA
+constexpr int kAttendDepth = RTP_ATTEND_DEPTH;           // cp.async stages per warp
 constexpr int kAttendCtasPerSm = 2;                      // resident attention CTAs per SM
 constexpr int kAttendThreads = kAttendWarps * 32;
 constexpr int kRowBytes = 128 * 2;                       // one K or V row
