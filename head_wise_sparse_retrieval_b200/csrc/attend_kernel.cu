@@ -33,7 +33,7 @@ constexpr int kTile = 16;
 constexpr int kDepth = kAttendDepth;
 constexpr int kWarpStage = 2 * kTile * kRowBytes;          // 16 K rows then 16 V rows
 constexpr int kOPitch = kHeadDim + 4;                      // padded row of the merge buffer
-constexpr int kCombFloats = kMaxGroup * kOPitch + kWarps * kMaxGroup * 2;
+constexpr int kCombFloats = kMaxGroup * kOPitch + kWarps * kMaxGroup * 2 + kMaxGroup * 2;
 constexpr int kMergeRows = kMergeThreads / 8;              // pieces a merge pass loads at once
 constexpr int kMergeRegs = 8;                              // passes kept in registers
 
@@ -156,24 +156,32 @@ __device__ __forceinline__ int tile_positions(const HeadRef& h, const LayerArgs&
 }
 
 // Gathers the tile's K and V rows into the stage: lane l copies 16-byte column c = l % 16 of
-// rows 2i + l / 16; the positions come from lanes 0..15 of pos.
+// rows 2i + l / 16; the positions come from lanes 0..15 of pos. A position outside [0, N) (a
+// corrupted list) is replaced by 0 and reported once per tile; rows past n are zero-filled.
 __device__ __forceinline__ void issue_tile(uint32_t stage, const HeadRef& h, int pos, int n,
                                            int lane, uint64_t policy, unsigned* status) {
   const int c = lane & 15, par = lane >> 4;
+  // swz(2i + par, c) = (2i + par) * 256 + ((c ^ ((2i + par) & 7)) << 4)
+  //                  = par * 256 + 512 i + (((c ^ par) ^ 2 (i & 3)) << 4)
+  const uint32_t lane_base = stage + (uint32_t)par * kRowBytes;
+  const int cx = c ^ par;
+  const __nv_bfloat16* kcol = h.kbase + c * 8;
+  const __nv_bfloat16* vcol = h.vbase + c * 8;
+  bool bad = false;
 #pragma unroll
   for (int i = 0; i < kTile / 2; ++i) {
     const int row = 2 * i + par;
-    int p = __shfl_sync(0xffffffffu, pos, row);
+    const int p = __shfl_sync(0xffffffffu, pos, row);
     const bool valid = row < n;
-    if (valid && (p < 0 || p >= h.N)) {
-      if (c == 0) atomicOr(status, kDevBadIndex);
-      p = 0;
-    }
-    const size_t off = valid ? (size_t)p * kHeadDim + c * 8 : 0;
+    const bool in = (unsigned)p < (unsigned)h.N;
+    bad |= valid && !in;
+    const size_t off = (valid && in) ? (size_t)p * kHeadDim : 0;
     const unsigned bytes = valid ? 16u : 0u;
-    cp_async_16(stage + swz(row, c), h.kbase + off, bytes, policy);
-    cp_async_16(stage + swz(kTile + row, c), h.vbase + off, bytes, policy);
+    const uint32_t dst = lane_base + 512u * i + ((uint32_t)(cx ^ (2 * (i & 3))) << 4);
+    cp_async_16(dst, kcol + off, bytes, policy);
+    cp_async_16(dst + kTile * kRowBytes, vcol + off, bytes, policy);
   }
+  if (__any_sync(0xffffffffu, bad) && lane == 0) atomicOr(status, kDevBadIndex);
 }
 
 }  // namespace
@@ -446,30 +454,46 @@ __global__ void __launch_bounds__(kAttendThreads, kAttendCtasPerSm) attend_kerne
     // it ends at the head's size; one piece covering both is the whole head
     const int len = (int)(sOff[hd + 1] - sOff[hd]);
     const bool first_piece = (r0 == 0), last_piece = (r1 == len);
-    float* out_h = a.out + ((size_t)b * a.Hq + (size_t)kvh * a.G) * kHeadDim;
     const bool single = first_piece && last_piece;
-    float* piece = w.partials + ((size_t)blockIdx.x + hd) * kPartFloats;
-    for (int jq = 0; jq < a.G; ++jq) {
+    float* sFin = sML + kWarps * kMaxGroup * 2;  // [8][2]: M, then L (1 / L for a whole head)
+    if (tid < a.G) {  // the piece's (M, L) per query head, over the warps
       float M = -INFINITY;
 #pragma unroll
-      for (int wq = 0; wq < kWarps; ++wq) M = fmaxf(M, sML[(wq * kMaxGroup + jq) * 2]);
+      for (int wq = 0; wq < kWarps; ++wq) M = fmaxf(M, sML[(wq * kMaxGroup + tid) * 2]);
       float L = 0.f;
 #pragma unroll
       for (int wq = 0; wq < kWarps; ++wq) {
-        const float mw = sML[(wq * kMaxGroup + jq) * 2];
-        if (mw != -INFINITY) L += sML[(wq * kMaxGroup + jq) * 2 + 1] * exp2f(mw - M);
+        const float mw = sML[(wq * kMaxGroup + tid) * 2];
+        if (mw != -INFINITY) L += sML[(wq * kMaxGroup + tid) * 2 + 1] * exp2f(mw - M);
       }
-      for (int d = tid; d < kHeadDim; d += kAttendThreads) {  // one output dimension per thread
-        const float O = sO[jq * kOPitch + d];
+      sFin[2 * tid] = M;
+      sFin[2 * tid + 1] = single ? 1.f / L : L;
+    }
+    __syncthreads();
+    // output or partial: thread tid writes query head tid / 16, dimensions 8 (tid % 16) .. +7
+    // (two 16-byte stores); with fewer than 128 threads the loop covers the rest
+    for (int e = tid; e < kMaxGroup * 16; e += kAttendThreads) {
+      const int jq = e >> 4, d0 = (e & 15) * 8;
+      if (jq < a.G) {
+        const float4* src = reinterpret_cast<const float4*>(sO + jq * kOPitch + d0);
+        float4 o0 = src[0], o1 = src[1];
+        float4* dst;
         if (single) {
-          out_h[(size_t)jq * kHeadDim + d] = O / L;
+          const float inv = sFin[2 * jq + 1];
+          o0.x *= inv; o0.y *= inv; o0.z *= inv; o0.w *= inv;
+          o1.x *= inv; o1.y *= inv; o1.z *= inv; o1.w *= inv;
+          dst = reinterpret_cast<float4*>(
+              a.out + ((size_t)b * a.Hq + (size_t)kvh * a.G + jq) * kHeadDim + d0);
         } else {
-          piece[jq * kHeadDim + d] = O;
-          if (d == 0) {
-            piece[kPartO + jq] = M;
-            piece[kPartO + kMaxGroup + jq] = L;
+          float* piece = w.partials + ((size_t)blockIdx.x + hd) * kPartFloats;
+          dst = reinterpret_cast<float4*>(piece + jq * kHeadDim + d0);
+          if ((e & 15) == 0) {
+            piece[kPartO + jq] = sFin[2 * jq];
+            piece[kPartO + kMaxGroup + jq] = sFin[2 * jq + 1];
           }
         }
+        dst[0] = o0;
+        dst[1] = o1;
       }
     }
     if (tid == 0) {  // merge_kernel reads the head's piece range (CTAs first .. last)
