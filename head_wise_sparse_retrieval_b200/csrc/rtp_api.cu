@@ -33,6 +33,14 @@ struct rtp_handle {
   cudaStream_t last_stream = nullptr;
   int last_nret = 0;
   short last_slot_of_kvh[kMaxKvHeads];
+  // rtp_decode_step_host replays the layer sequence as a CUDA graph, captured once per
+  // (layer count, p, cache pointers, masks) on a stream of the handle
+  cudaStream_t cap_stream = nullptr;
+  cudaGraphExec_t step_exec = nullptr;
+  int step_layers = 0;
+  float step_p = 0.f;
+  std::vector<const void*> step_ptrs;
+  std::vector<uint8_t> step_masks;
   // kernel profiling (rtp_profile_enable)
   bool prof = false;
   std::vector<cudaEvent_t> prof_ev;   // 2 per launch
@@ -395,6 +403,8 @@ rtp_status rtp_destroy(rtp_handle* h) {
   DeviceGuard guard(h->device);
   cudaDeviceSynchronize();
   for (cudaEvent_t ev : h->prof_ev) cudaEventDestroy(ev);
+  if (h->step_exec) cudaGraphExecDestroy(h->step_exec);
+  if (h->cap_stream) cudaStreamDestroy(h->cap_stream);
 
   cudaError_t e = cudaFree(h->ws_mem);
   delete h;
@@ -471,20 +481,72 @@ rtp_status rtp_decode_step_host(rtp_handle* h, int num_layers, const void* q_hos
   if (e == cudaSuccess)
     e = cudaMemcpyAsync(h->stage_seq, seq_lens_host, B * 4, cudaMemcpyHostToDevice, s);
   if (e != cudaSuccess) return cuda_fail(e, "host-to-device copy");
-  for (int l = 0; l < num_layers; ++l) {
-    rtp_layer_io io;
-    memset(&io, 0, sizeof io);
-    io.q = static_cast<const char*>(h->stage_q) + (size_t)l * q_layer * 2;
-    io.q_idx = static_cast<const char*>(h->stage_qidx) + (size_t)l * qi_layer * 2;
-    io.k_cache = k_cache[l];
-    io.v_cache = v_cache[l];
-    io.k_idx = k_idx ? k_idx[l] : nullptr;
-    io.seq_lens = h->stage_seq;
-    io.retrieval_mask = masks + (size_t)l * c.num_kv_heads;
-    io.top_p = top_p;
-    io.out = h->stage_out + (size_t)l * q_layer;
-    rtp_status st = rtp_decode_step(h, l, &io, stream);
+  // the layers read and write only the staging buffers and the caller's caches, so the launch
+  // sequence is the same from call to call while the pointers, masks and p are
+  auto enqueue_all = [&](cudaStream_t st_stream) -> rtp_status {
+    for (int l = 0; l < num_layers; ++l) {
+      rtp_layer_io io;
+      memset(&io, 0, sizeof io);
+      io.q = static_cast<const char*>(h->stage_q) + (size_t)l * q_layer * 2;
+      io.q_idx = static_cast<const char*>(h->stage_qidx) + (size_t)l * qi_layer * 2;
+      io.k_cache = k_cache[l];
+      io.v_cache = v_cache[l];
+      io.k_idx = k_idx ? k_idx[l] : nullptr;
+      io.seq_lens = h->stage_seq;
+      io.retrieval_mask = masks + (size_t)l * c.num_kv_heads;
+      io.top_p = top_p;
+      io.out = h->stage_out + (size_t)l * q_layer;
+      rtp_status st = rtp_decode_step(h, l, &io, st_stream);
+      if (st != RTP_OK) return st;
+    }
+    return RTP_OK;
+  };
+  if (h->prof) {  // profiling events cannot sit in a graph: launch eagerly
+    rtp_status st = enqueue_all(s);
     if (st != RTP_OK) return st;
+  } else {
+    std::vector<const void*> ptrs(3 * L);
+    for (size_t l = 0; l < L; ++l) {
+      ptrs[3 * l] = k_cache[l];
+      ptrs[3 * l + 1] = v_cache[l];
+      ptrs[3 * l + 2] = k_idx ? k_idx[l] : nullptr;
+    }
+    std::vector<uint8_t> mk(masks, masks + L * c.num_kv_heads);
+    const bool reuse = h->step_exec && h->step_layers == num_layers && h->step_p == top_p &&
+                       h->step_ptrs == ptrs && h->step_masks == mk;
+    if (!reuse) {
+      if (h->step_exec) {
+        cudaGraphExecDestroy(h->step_exec);
+        h->step_exec = nullptr;
+      }
+      if (!h->cap_stream) {
+        e = cudaStreamCreateWithFlags(&h->cap_stream, cudaStreamNonBlocking);
+        if (e != cudaSuccess) return cuda_fail(e, "cudaStreamCreate");
+      }
+      e = cudaStreamBeginCapture(h->cap_stream, cudaStreamCaptureModeThreadLocal);
+      if (e != cudaSuccess) return cuda_fail(e, "cudaStreamBeginCapture");
+      rtp_status st = enqueue_all(h->cap_stream);
+      cudaGraph_t graph = nullptr;
+      e = cudaStreamEndCapture(h->cap_stream, &graph);
+      if (st != RTP_OK) {
+        if (graph) cudaGraphDestroy(graph);
+        return st;
+      }
+      if (e != cudaSuccess) return cuda_fail(e, "cudaStreamEndCapture");
+      e = cudaGraphInstantiate(&h->step_exec, graph, 0);
+      cudaGraphDestroy(graph);
+      if (e != cudaSuccess) {
+        h->step_exec = nullptr;
+        return cuda_fail(e, "cudaGraphInstantiate");
+      }
+      h->step_layers = num_layers;
+      h->step_p = top_p;
+      h->step_ptrs = std::move(ptrs);
+      h->step_masks = std::move(mk);
+    }
+    e = cudaGraphLaunch(h->step_exec, s);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaGraphLaunch");
+    h->last_stream = s;
   }
   e = cudaMemcpyAsync(out_host, h->stage_out, L * q_layer * 4, cudaMemcpyDeviceToHost, s);
   if (e != cudaSuccess) return cuda_fail(e, "device-to-host copy");

@@ -140,7 +140,11 @@ RTP_API rtp_status rtp_dense_decode(rtp_handle *h, const rtp_layer_io *io, void 
  * masks[l * Hkv ...], and copies the fp32 outputs back into out_host ([L][B][Hq][D]).
  * Host buffers should be pinned for the copies to be asynchronous. Synchronises `stream`
  * before returning (the outputs are in out_host on return). Staging is allocated by
- * rtp_create for cfg.num_layers layers. Errors as rtp_decode_step. */
+ * rtp_create for cfg.num_layers layers. The layer launches are captured once into a CUDA
+ * graph on a stream of the handle (created on first use) and replayed on `stream` while
+ * num_layers, top_p, the cache pointers and the masks stay the same; a change re-captures.
+ * While profiling is enabled the layers are launched one by one instead. Must not be called
+ * while `stream` is being captured. Errors as rtp_decode_step. */
 RTP_API rtp_status rtp_decode_step_host(rtp_handle *h, int num_layers, const void *q_host,
                                 const void *q_idx_host, const int32_t *seq_lens_host,
                                 const void *const *k_cache, const void *const *v_cache,

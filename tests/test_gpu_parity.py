@@ -191,10 +191,30 @@ def test_host_buffer_entry_matches_device_entry():
         qi = torch.stack([li.q_idx for li in lis]).cpu().pin_memory()
         seq = lis[0].seq_lens.cpu().pin_memory()
         out = torch.empty((2,) + tuple(dev_out[0].shape), dtype=torch.float32).pin_memory()
-        h.decode_step_host(q, qi, seq, [rtp.layer_from(li) for li in lis], p.retrieval,
-                           p.top_p, out)
-    for l in range(2):
-        assert torch.equal(out[l], dev_out[l].cpu())
+        views = [rtp.layer_from(li) for li in lis]
+        h.decode_step_host(q, qi, seq, views, p.retrieval, p.top_p, out)
+        for l in range(2):
+            assert torch.equal(out[l], dev_out[l].cpu())
+        # a second call replays the captured launches on new queries from the same staging
+        for li in lis:
+            li.q.neg_()
+        dev_out2 = [run_layer(h, p, li, l)[0] for l, li in enumerate(lis)]
+        q2 = torch.stack([li.q for li in lis]).cpu().pin_memory()
+        h.decode_step_host(q2, qi, seq, views, p.retrieval, p.top_p, out)
+        for l in range(2):
+            assert torch.equal(out[l], dev_out2[l].cpu())
+            assert not torch.equal(dev_out2[l], dev_out[l])
+        # other masks: the launches are captured again
+        masks = p.retrieval.copy()
+        masks[0] = 1 - masks[0]
+        dev_out3 = []
+        for l, li in enumerate(lis):
+            o = torch.empty_like(dev_out2[l])
+            h.decode_step(l, rtp.layer_from(li), masks[l], p.top_p, o)
+            dev_out3.append(o)
+        h.decode_step_host(q2, qi, seq, views, masks, p.top_p, out)
+        for l in range(2):
+            assert torch.equal(out[l], dev_out3[l].cpu())
 
 
 def test_bad_seq_len_is_reported_not_faulted():
