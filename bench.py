@@ -268,6 +268,8 @@ def main():
     ap.add_argument("--ctx", type=int, default=None, help="other context length (debug only)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-dense", action="store_true")
+    ap.add_argument("--p-sweep", default="0.8,0.95",
+                    help="other top-p values timed the same way (comma list; empty: none)")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--single-layer", type=int, default=None,
                     help="profiling case: only this layer of the workload, decoded --reps times")
@@ -397,6 +399,44 @@ def main():
     if hashlib.sha256(open(src, "rb").read()).hexdigest()[:16] == ATTEND_NCU["source_sha256_16"]:
         traffic = att_bytes_per_launch * ATTEND_NCU["traffic_bytes"] / ATTEND_NCU["algorithmic_bytes"]
 
+    # the same step at other p (the 1M-context configuration sweeps p over 0.8 / 0.9 / 0.95)
+    p_sweep = {}
+    for ps in [x for x in args.p_sweep.split(",") if x.strip()]:
+        pv = float(ps)
+        with torch.cuda.stream(stream):
+            for l in range(L):
+                h.decode_step(l, views[l], plan.retrieval[l], pv, outs[l], cnts[l], stream=stream)
+        torch.cuda.synchronize()
+        sel_p = [c.cpu().numpy() for c in cnts]
+        bytes_p = step_bytes(plan, sel_p)[0]
+        gp = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(gp, stream=stream):
+            for l in range(L):
+                h.decode_step(l, views[l], plan.retrieval[l], pv, outs[l], cnts[l], stream=stream)
+        with torch.cuda.stream(stream):
+            for _ in range(args.warmup):
+                gp.replay()
+        torch.cuda.synchronize()
+        p0 = torch.cuda.Event(enable_timing=True)
+        p1 = torch.cuda.Event(enable_timing=True)
+        if world > 1:
+            dist.barrier()
+        with torch.cuda.stream(stream):
+            p0.record(stream)
+            for _ in range(args.steps):
+                gp.replay()
+            p1.record(stream)
+        torch.cuda.synchronize()
+        pms = max_over_ranks(p0.elapsed_time(p1) / args.steps, world, dev)
+        n_p = [int(x[b, k]) for l, x in enumerate(sel_p) for b in range(B) for k in range(Hkv)
+               if plan.retrieval[l, k]]
+        p_sweep[ps.strip()] = {"ms_per_step": pms, "steps_per_s": throughput(world, pms),
+                               "effective_gbs": bytes_p / (pms * 1e-3) / 1e9,
+                               "roofline_frac_step": bytes_p / (pms * 1e-3) / 1e9 / hbm,
+                               "algorithmic_bytes_per_step": bytes_p,
+                               "mean_selected": float(np.mean(n_p)) if n_p else 0.0}
+        del gp
+
     # dense decode on the same caches (the speedup denominator)
     dense = None
     if not args.no_dense:
@@ -493,6 +533,7 @@ def main():
         "selection": {"retrieval_heads": len(n_sel),
                       "mean_selected": float(np.mean(n_sel)) if n_sel else 0.0,
                       "max_selected": int(max(n_sel)) if n_sel else 0},
+        "p_sweep": p_sweep,
         "dense": dense,
         "e2e": e2e,
         "cpu_baseline": cpu,
