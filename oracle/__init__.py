@@ -36,6 +36,7 @@ class _LayerCfg(ctypes.Structure):
         ("max_ctx", ctypes.c_int64), ("window", ctypes.c_int64), ("sinks", ctypes.c_int64),
         ("idx_range", ctypes.c_double), ("idx_scale", ctypes.c_double),
         ("attn_scale", ctypes.c_double), ("top_p", ctypes.c_double),
+        ("top_k", ctypes.c_int64),
     ]
 
 
@@ -53,6 +54,9 @@ def lib():
         L.orc_hist_topp.argtypes = [_dp, ctypes.c_int64, ctypes.c_double, ctypes.c_double,
                                     ctypes.c_int, _ip, _dp, _dp, _ip, _i64p, _i64p]
         L.orc_exact_topp.argtypes = [_dp, ctypes.c_int64, ctypes.c_double, _i64p, _i64p]
+        L.orc_hist_topk.argtypes = [_dp, ctypes.c_int64, ctypes.c_int64, ctypes.c_double,
+                                    ctypes.c_int, _ip, _i64p, _i64p, _ip, _i64p, _i64p]
+        L.orc_exact_topk.argtypes = [_dp, ctypes.c_int64, ctypes.c_int64, _i64p, _i64p]
         L.orc_window_sink_set.argtypes = [ctypes.c_int64, ctypes.c_int64, ctypes.c_int64,
                                           _i64p, _i64p]
         L.orc_sparse_attention.argtypes = [_u16p, _u16p, _u16p, _i64p, ctypes.c_int64,
@@ -140,6 +144,40 @@ def exact_topp(s, p: float) -> np.ndarray:
     return sel[: nsel.value].copy()
 
 
+@dataclass
+class HistTopK:
+    sel: np.ndarray      # ascending token positions with bin >= b*
+    bstar: int
+    bins: np.ndarray     # bin of every token
+    count: np.ndarray    # K_b, tokens per bin
+    suffix: np.ndarray   # N_b, tokens in bins >= b
+
+
+def hist_topk(s, k: int, range_: float = 16.0, nbins: int = 256) -> HistTopK:
+    s = np.ascontiguousarray(s, dtype=np.float64)
+    n = s.shape[0]
+    bins = np.empty(n, np.int32)
+    count = np.empty(nbins, np.int64)
+    suffix = np.empty(nbins, np.int64)
+    sel = np.empty(n, np.int64)
+    bstar = ctypes.c_int()
+    nsel = ctypes.c_int64()
+    _check(lib().orc_hist_topk(_ptr(s, ctypes.c_double), n, int(k), float(range_), nbins,
+                               _ptr(bins, ctypes.c_int), _ptr(count, ctypes.c_int64),
+                               _ptr(suffix, ctypes.c_int64), ctypes.byref(bstar),
+                               _ptr(sel, ctypes.c_int64), ctypes.byref(nsel)), "hist_topk")
+    return HistTopK(sel[: nsel.value].copy(), bstar.value, bins, count, suffix)
+
+
+def exact_topk(s, k: int) -> np.ndarray:
+    s = np.ascontiguousarray(s, dtype=np.float64)
+    sel = np.empty(s.shape[0], np.int64)
+    nsel = ctypes.c_int64()
+    _check(lib().orc_exact_topk(_ptr(s, ctypes.c_double), s.shape[0], int(k),
+                                _ptr(sel, ctypes.c_int64), ctypes.byref(nsel)), "exact_topk")
+    return sel[: nsel.value].copy()
+
+
 def window_sink_set(n_tok: int, window: int = 8192, sinks: int = 4) -> np.ndarray:
     sel = np.empty(n_tok, np.int64)
     nsel = ctypes.c_int64()
@@ -168,6 +206,7 @@ def sparse_attention(q, k, v, idx, scale: float | None = None) -> np.ndarray:
 
 
 def decode_layer(*, q, q_idx, k_cache, v_cache, k_idx, seq_lens, retrieval_mask, top_p: float,
+                 top_k: int = 0,
                  mode: int = MODE_HIST, window: int = 8192, sinks: int = 4, num_bins: int = 256,
                  idx_range: float = 16.0, idx_scale: float = 0.25, attn_scale: float | None = None,
                  num_threads: int | None = None):
@@ -187,7 +226,7 @@ def decode_layer(*, q, q_idx, k_cache, v_cache, k_idx, seq_lens, retrieval_mask,
         R = 16
     cfg = _LayerCfg(B, Hq, Hkv, D, R, num_bins, Nmax, window, sinks, float(idx_range),
                     float(idx_scale), float(1.0 / np.sqrt(D) if attn_scale is None else attn_scale),
-                    float(top_p))
+                    float(top_p), int(top_k))
     seq = np.ascontiguousarray(seq_lens, dtype=np.int64)
     mask = np.ascontiguousarray(retrieval_mask, dtype=np.uint8)
     assert seq.shape == (B,) and mask.shape == (Hkv,)
@@ -211,6 +250,7 @@ def max_threads() -> int:
 
 __all__ = [
     "MODE_HIST", "MODE_EXACT", "MODE_DENSE", "bf16_to_f64", "f16_to_f64", "indexer_scores",
-    "hist_topp", "HistSelection", "exact_topp", "window_sink_set", "sparse_attention",
+    "hist_topp", "HistSelection", "exact_topp", "hist_topk", "HistTopK", "exact_topk",
+    "window_sink_set", "sparse_attention",
     "decode_layer", "max_threads",
 ]

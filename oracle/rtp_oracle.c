@@ -32,6 +32,9 @@
  *   - C_b = sum of the masses of bins b..nbins-1, accumulated from the top bin down;
  *     b* is the highest b with C_b >= p * C_0; the selection is every token with bin >= b*;
  *   - the G query heads of a GQA group share their KV head's selection;
+ *   - fixed top-k through the same histogram (the top-k / top-p comparison of [P1] section 三
+ *     "洞察 3: 动态 Top-P 选择", top-2k / 4k / 16k): b* is the highest b whose suffix COUNT
+ *     N_b = #{n : bin(n) >= b} reaches k (b* = 0, every token, when k >= n_tok);
  *   - a local head attends over {0..sinks-1} U {N-window..N-1} (set union, positions
  *     clipped to [0, N)); the cache already holds the current token at position N-1.
  *
@@ -167,6 +170,72 @@ int orc_hist_topp(const double *s, int64_t n_tok, double p, double range, int nb
     return ORC_OK;
 }
 
+/* ---- fixed top-k through the same histogram [P1 洞察 3, top-k vs top-p] ---------------- */
+
+/*
+ * Histogram top-k of the scores s[0..n_tok), k >= 1. The bins are those of orc_hist_topp:
+ *   bin(n)  = clamp(floor((s_n - (s_max - range)) * nbins / range), 0, nbins - 1)
+ *   K_b     = #{n : bin(n) = b}          (count of bin b)
+ *   N_b     = K_{nbins-1} + ... + K_b    (accumulated from the top bin down)
+ *   b*      = max{ b : N_b >= k }, or 0 if no bin reaches k (k > n_tok)
+ *   S       = { n : bin(n) >= b* }, listed ascending.
+ * Optional outputs (may be NULL): bin[n_tok], count[nbins], suffix[nbins] (N_b).
+ */
+int orc_hist_topk(const double *s, int64_t n_tok, int64_t k, double range, int nbins,
+                  int *bin, int64_t *count, int64_t *suffix, int *bstar, int64_t *sel,
+                  int64_t *n_sel)
+{
+    if (!s || !bstar || !sel || !n_sel || n_tok <= 0 || nbins <= 0 || !(range > 0.0) || k < 1)
+        return ORC_ERR_ARG;
+
+    double s_max = s[0];
+    for (int64_t n = 1; n < n_tok; n++)
+        if (s[n] > s_max)
+            s_max = s[n];
+    double lo = s_max - range;
+
+    int *b_of = (int *)malloc(sizeof(int) * (size_t)n_tok);
+    int64_t *K = (int64_t *)calloc((size_t)nbins, sizeof(int64_t));
+    int64_t *Nb = (int64_t *)calloc((size_t)nbins, sizeof(int64_t));
+    if (!b_of || !K || !Nb) {
+        free(b_of); free(K); free(Nb);
+        return ORC_ERR_NOMEM;
+    }
+    for (int64_t n = 0; n < n_tok; n++) {
+        double x = floor((s[n] - lo) * (double)nbins / range);
+        int b = x < 0.0 ? 0 : (x > (double)(nbins - 1) ? nbins - 1 : (int)x);
+        b_of[n] = b;
+        K[b] += 1;
+    }
+    int64_t acc = 0;
+    for (int b = nbins - 1; b >= 0; b--) {
+        acc += K[b];
+        Nb[b] = acc;
+    }
+    int bs = 0;
+    for (int b = nbins - 1; b >= 0; b--) {
+        if (Nb[b] >= k) {
+            bs = b;
+            break;
+        }
+    }
+    int64_t m = 0;
+    for (int64_t n = 0; n < n_tok; n++)
+        if (b_of[n] >= bs)
+            sel[m++] = n;
+
+    *bstar = bs;
+    *n_sel = m;
+    if (bin)
+        memcpy(bin, b_of, sizeof(int) * (size_t)n_tok);
+    if (count)
+        memcpy(count, K, sizeof(int64_t) * (size_t)nbins);
+    if (suffix)
+        memcpy(suffix, Nb, sizeof(int64_t) * (size_t)nbins);
+    free(b_of); free(K); free(Nb);
+    return ORC_OK;
+}
+
 /* ---- exact (sort-based) top-p, the definition the histogram approximates ------------ */
 
 typedef struct {
@@ -224,6 +293,29 @@ int orc_exact_topp(const double *s, int64_t n_tok, double p, int64_t *sel, int64
     qsort(sel, (size_t)k, sizeof(int64_t), orc_cmp_i64);
     *n_sel = k;
     free(v); free(cum);
+    return ORC_OK;
+}
+
+/* The k highest scores (ties by ascending position; every token when k >= n_tok), returned
+ * ascending: the exact selection the histogram top-k approximates. */
+int orc_exact_topk(const double *s, int64_t n_tok, int64_t k, int64_t *sel, int64_t *n_sel)
+{
+    if (!s || !sel || !n_sel || n_tok <= 0 || k < 1)
+        return ORC_ERR_ARG;
+    orc_scored *v = (orc_scored *)malloc(sizeof(orc_scored) * (size_t)n_tok);
+    if (!v)
+        return ORC_ERR_NOMEM;
+    for (int64_t n = 0; n < n_tok; n++) {
+        v[n].s = s[n];
+        v[n].n = n;
+    }
+    qsort(v, (size_t)n_tok, sizeof(orc_scored), orc_cmp_desc);
+    int64_t m = k < n_tok ? k : n_tok;
+    for (int64_t i = 0; i < m; i++)
+        sel[i] = v[i].n;
+    qsort(sel, (size_t)m, sizeof(int64_t), orc_cmp_i64);
+    *n_sel = m;
+    free(v);
     return ORC_OK;
 }
 
@@ -303,6 +395,7 @@ typedef struct {
     int batch, num_q_heads, num_kv_heads, head_dim, idx_dim, num_bins;
     int64_t max_ctx, window, sinks;
     double idx_range, idx_scale, attn_scale, top_p;
+    int64_t top_k;  /* > 0: retrieval heads keep the histogram (or exact) top-k, not top-p */
 } orc_layer_cfg;
 
 enum { ORC_MODE_HIST = 0, ORC_MODE_EXACT = 1, ORC_MODE_DENSE = 2 };
@@ -361,10 +454,16 @@ int orc_decode_layer(const orc_layer_cfg *c, int mode, const uint16_t *q, const 
                 } else {
                     rc = orc_indexer_scores(q_idx + head * R, k_idx + head * Nmax * R, N, R,
                                             c->idx_scale, s);
-                    if (rc == ORC_OK && mode == ORC_MODE_HIST) {
+                    if (rc == ORC_OK && mode == ORC_MODE_HIST && c->top_k > 0) {
+                        int bs;
+                        rc = orc_hist_topk(s, N, c->top_k, c->idx_range, c->num_bins, NULL,
+                                           NULL, NULL, &bs, sel, &k);
+                    } else if (rc == ORC_OK && mode == ORC_MODE_HIST) {
                         int bs;
                         rc = orc_hist_topp(s, N, c->top_p, c->idx_range, c->num_bins, NULL,
                                            NULL, NULL, &bs, sel, &k);
+                    } else if (rc == ORC_OK && c->top_k > 0) {
+                        rc = orc_exact_topk(s, N, c->top_k, sel, &k);
                     } else if (rc == ORC_OK) {
                         rc = orc_exact_topp(s, N, c->top_p, sel, &k);
                     }

@@ -209,6 +209,99 @@ def test_hist_brute_force_tiny(orc):
 
 # ---- window + sinks --------------------------------------------------------------------
 
+# ---- fixed top-k through the histogram --------------------------------------------------
+
+def test_hist_topk_golden_counts(orc):
+    g = _golden("hist_topk_counts.json")
+    s = np.array(g["scores"])
+    for case in g["cases"]:
+        h = orc.hist_topk(s, case["k"])
+        assert list(h.bins) == g["bins"]
+        assert h.bstar == case["bstar"], case
+        assert list(h.sel) == case["sel"], case
+
+
+def _check_topk_invariants(orc, s, k):
+    h = orc.hist_topk(s, k)
+    n = s.size
+    inset = np.zeros(n, bool)
+    inset[h.sel] = True
+    assert np.array_equal(inset, h.bins >= h.bstar)          # upward closed in bins
+    assert h.sel.size >= min(k, n)                             # reaches k
+    if k <= n:
+        # closed form: b* is the bin of the k-th highest score (ties by position), found
+        # here by sorting, not by the suffix counts
+        kth = np.lexsort((np.arange(n), -s))[k - 1]
+        assert h.bstar == h.bins[kth]
+        # minimal: the bins strictly above b* hold fewer than k tokens
+        assert int((h.bins > h.bstar).sum()) < k
+    else:
+        assert h.sel.size == n
+    # superset of the exact top-k; the surplus lies inside bin b*
+    ex = orc.exact_topk(s, k)
+    assert ex.size == min(k, n) and inset[ex].all()
+    assert np.all(h.bins[~np.isin(np.arange(n), ex) & inset] == h.bstar)
+    assert np.array_equal(h.suffix, np.cumsum(h.count[::-1])[::-1])
+    return h
+
+
+@pytest.mark.parametrize("sigma", [0.05, 0.5, 2.39, 12.0])
+@pytest.mark.parametrize("k", [1, 2, 17, 2048, 4096, 16384, 50000])
+def test_hist_topk_invariants_random(orc, sigma, k):
+    rng = np.random.default_rng([int(sigma * 100), k])
+    _check_topk_invariants(orc, rng.normal(0, sigma, 20000), k)
+
+
+def test_hist_topk_ties_and_degenerate(orc):
+    s = np.zeros(50)                                   # all tied: one bin holds everything
+    for k in (1, 7, 50, 51):
+        h = _check_topk_invariants(orc, s, k)
+        assert h.sel.size == 50 and h.bstar == (255 if k <= 50 else 0)
+    s = np.array([3.0])
+    assert orc.hist_topk(s, 1).sel.tolist() == [0]
+    with pytest.raises(RuntimeError):
+        orc.hist_topk(np.array([1.0, 2.0]), 0)
+
+
+def test_exact_topk_brute_force_tiny(orc):
+    rng = np.random.default_rng(17)
+    for trial in range(40):
+        n = int(rng.integers(1, 8))
+        s = np.round(rng.normal(0, 1, n), 1)             # rounded: ties occur
+        for k in range(1, n + 2):
+            got = orc.exact_topk(s, k)
+            m = min(k, n)
+            # the k-subset whose members all beat every non-member in (score, -position)
+            best = None
+            for sub in itertools.combinations(range(n), m):
+                rest = [j for j in range(n) if j not in sub]
+                if all((s[i], -i) > (s[j], -j) for i in sub for j in rest):
+                    best = sub
+            assert best is not None and got.tolist() == list(best)
+
+
+def test_layer_topk_equals_attention_over_hist_topk(orc):
+    from head_wise_sparse_retrieval_b200 import workloads as W
+    p = W.custom(batch=2, num_q_heads=16, num_kv_heads=2, seq_lens=[3000, 700], max_ctx=3000,
+                 retrieval=[1, 0], kinds=[[W.KIND_DIFFUSE, 0]] * 2, seed=8)
+    _, li, io = _layer(p)
+    out, nsel = orc.decode_layer(**io, top_p=0.9, top_k=256)
+    for b in range(2):
+        N = int(io["seq_lens"][b])
+        s = orc.indexer_scores(io["q_idx"][b, 0], io["k_idx"][b, 0, :N])
+        sel = orc.hist_topk(s, 256).sel
+        assert nsel[b, 0] == sel.size >= 256
+        ref = orc.sparse_attention(io["q"][b, :8], io["k_cache"][b, 0], io["v_cache"][b, 0], sel)
+        assert np.allclose(out[b, :8], ref, rtol=1e-12, atol=1e-14)
+    # k at or above N is dense attention
+    dense, _ = orc.decode_layer(**io, top_p=0.9, mode=orc.MODE_DENSE)
+    allk, _ = orc.decode_layer(**io, top_p=0.9, top_k=3000)
+    assert np.allclose(allk[:, :8], dense[:, :8], rtol=1e-12, atol=1e-13)
+    # the exact mode keeps exactly k
+    _, n_ex = orc.decode_layer(**io, top_p=0.9, top_k=256, mode=orc.MODE_EXACT)
+    assert n_ex[0, 0] == 256 and n_ex[1, 0] == 256
+
+
 def test_window_sink_golden(orc):
     g = _golden("window_sink_sets.json")
     for c in g["cases"]:
