@@ -270,6 +270,8 @@ def main():
     ap.add_argument("--no-dense", action="store_true")
     ap.add_argument("--p-sweep", default="0.8,0.95",
                     help="other top-p values timed the same way (comma list; empty: none)")
+    ap.add_argument("--k-sweep", default="2048,4096,16384",
+                    help="fixed top-k values (through the same histogram) timed the same way")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--single-layer", type=int, default=None,
                     help="profiling case: only this layer of the workload, decoded --reps times")
@@ -400,42 +402,48 @@ def main():
         traffic = att_bytes_per_launch * ATTEND_NCU["traffic_bytes"] / ATTEND_NCU["algorithmic_bytes"]
 
     # the same step at other p (the 1M-context configuration sweeps p over 0.8 / 0.9 / 0.95)
-    p_sweep = {}
-    for ps in [x for x in args.p_sweep.split(",") if x.strip()]:
-        pv = float(ps)
+    # and with the fixed top-k of the pages' top-k / top-p comparison (2k / 4k / 16k)
+    def time_variant(pv, kv):
+        def run():
+            for l in range(L):
+                h.decode_step(l, views[l], plan.retrieval[l], pv, outs[l], cnts[l],
+                              stream=stream, top_k=kv)
         with torch.cuda.stream(stream):
-            for l in range(L):
-                h.decode_step(l, views[l], plan.retrieval[l], pv, outs[l], cnts[l], stream=stream)
+            run()
         torch.cuda.synchronize()
-        sel_p = [c.cpu().numpy() for c in cnts]
-        bytes_p = step_bytes(plan, sel_p)[0]
-        gp = torch.cuda.CUDAGraph()
-        with torch.cuda.graph(gp, stream=stream):
-            for l in range(L):
-                h.decode_step(l, views[l], plan.retrieval[l], pv, outs[l], cnts[l], stream=stream)
+        sel_v = [c.cpu().numpy() for c in cnts]
+        bytes_v = step_bytes(plan, sel_v)[0]
+        gv = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(gv, stream=stream):
+            run()
         with torch.cuda.stream(stream):
             for _ in range(args.warmup):
-                gp.replay()
+                gv.replay()
         torch.cuda.synchronize()
-        p0 = torch.cuda.Event(enable_timing=True)
-        p1 = torch.cuda.Event(enable_timing=True)
+        v0 = torch.cuda.Event(enable_timing=True)
+        v1 = torch.cuda.Event(enable_timing=True)
         if world > 1:
             dist.barrier()
         with torch.cuda.stream(stream):
-            p0.record(stream)
+            v0.record(stream)
             for _ in range(args.steps):
-                gp.replay()
-            p1.record(stream)
+                gv.replay()
+            v1.record(stream)
         torch.cuda.synchronize()
-        pms = max_over_ranks(p0.elapsed_time(p1) / args.steps, world, dev)
-        n_p = [int(x[b, k]) for l, x in enumerate(sel_p) for b in range(B) for k in range(Hkv)
+        vms = max_over_ranks(v0.elapsed_time(v1) / args.steps, world, dev)
+        n_v = [int(x[b, k]) for l, x in enumerate(sel_v) for b in range(B) for k in range(Hkv)
                if plan.retrieval[l, k]]
-        p_sweep[ps.strip()] = {"ms_per_step": pms, "steps_per_s": throughput(world, pms),
-                               "effective_gbs": bytes_p / (pms * 1e-3) / 1e9,
-                               "roofline_frac_step": bytes_p / (pms * 1e-3) / 1e9 / hbm,
-                               "algorithmic_bytes_per_step": bytes_p,
-                               "mean_selected": float(np.mean(n_p)) if n_p else 0.0}
-        del gp
+        del gv
+        return {"ms_per_step": vms, "steps_per_s": throughput(world, vms),
+                "effective_gbs": bytes_v / (vms * 1e-3) / 1e9,
+                "roofline_frac_step": bytes_v / (vms * 1e-3) / 1e9 / hbm,
+                "algorithmic_bytes_per_step": bytes_v,
+                "mean_selected": float(np.mean(n_v)) if n_v else 0.0}
+
+    p_sweep = {ps.strip(): time_variant(float(ps), 0)
+               for ps in args.p_sweep.split(",") if ps.strip()}
+    k_sweep = {ks.strip(): time_variant(plan.top_p, int(ks))
+               for ks in args.k_sweep.split(",") if ks.strip()}
 
     # dense decode on the same caches (the speedup denominator)
     dense = None
@@ -534,6 +542,7 @@ def main():
                       "mean_selected": float(np.mean(n_sel)) if n_sel else 0.0,
                       "max_selected": int(max(n_sel)) if n_sel else 0},
         "p_sweep": p_sweep,
+        "k_sweep": k_sweep,
         "dense": dense,
         "e2e": e2e,
         "cpu_baseline": cpu,

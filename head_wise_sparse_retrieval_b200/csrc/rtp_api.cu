@@ -23,6 +23,7 @@ struct rtp_handle {
   void* ws_mem = nullptr;
   size_t ws_bytes = 0;
   Workspace ws{};
+  unsigned* hist_cnt = nullptr;  // selection token counts per bin (fixed top-k)
   // staging for rtp_decode_step_host
   void* stage_q = nullptr;
   void* stage_qidx = nullptr;
@@ -130,6 +131,7 @@ WsPlan plan_workspace(const rtp_config* c, int attend_grid, int select_grid) {
       slots * 8,                             // 13 head_pieces
       ((size_t)attend_grid + slots) * kPartFloats * 4,  // 14 partials
       256,                                   // 15 status
+      (size_t)kHistCopies * slots * kBins * 4,  // 16 hist_cnt
   };
   WsPlan p{};
   size_t at = 0;
@@ -173,7 +175,8 @@ rtp_status check_io(const rtp_handle* h, const rtp_layer_io* io, bool need_idx) 
       return fail(RTP_ERR_INVALID_ARG, "q_idx and k_idx are required for retrieval heads");
     if (!aligned16(io->q_idx) || !aligned16(io->k_idx))
       return fail(RTP_ERR_INVALID_ARG, "q_idx and k_idx must be 16-byte aligned");
-    if (!(io->top_p > 0.f && io->top_p <= 1.f))
+    if (io->top_k < 0) return fail(RTP_ERR_INVALID_ARG, "top_k must be >= 0");
+    if (io->top_k == 0 && !(io->top_p > 0.f && io->top_p <= 1.f))
       return fail(RTP_ERR_INVALID_ARG, "top_p must be in (0, 1]");
   }
   (void)h;
@@ -223,14 +226,17 @@ cudaError_t launch_one(rtp_handle* h, int kind, Kernel k, dim3 grid, dim3 block,
   return e;
 }
 
-rtp_status enqueue_layer(rtp_handle* h, const LayerArgs& a0, cudaStream_t s) {
+rtp_status enqueue_layer(rtp_handle* h, const LayerArgs& a0, cudaStream_t s, int top_k = 0) {
   cudaError_t e;
   if (!a0.dense && a0.nret > 0) {
+    SelectArgs x;
+    x.top_k = top_k;
+    x.hist_cnt = h->hist_cnt;
     // the ranges are at most ceil(B * nret * max_ctx / grid) tokens: on chip when that fits
     const long long worst = (long long)a0.B * a0.nret * a0.max_ctx;
     const bool fits = (worst + h->select_grid - 1) / h->select_grid <= kScoreCap;
     e = launch_one(h, 0, fits ? select_kernel_onchip : select_kernel_spill, dim3(h->select_grid),
-                   dim3(kSelThreads), h->select_smem, s, true, a0, h->ws);
+                   dim3(kSelThreads), h->select_smem, s, true, a0, h->ws, x);
     if (e != cudaSuccess) return cuda_fail(e, "select_kernel launch");
   }
   const LayerArgs& a = a0;
@@ -371,6 +377,7 @@ rtp_status rtp_create(const rtp_config* cfg, int device, rtp_handle** out) {
   w.head_pieces = reinterpret_cast<int2*>(base + p.off[13]);
   w.partials = reinterpret_cast<float*>(base + p.off[14]);
   w.status = reinterpret_cast<unsigned*>(base + p.off[15]);
+  h->hist_cnt = reinterpret_cast<unsigned*>(base + p.off[16]);
   w.ld = (int)round_up((size_t)cfg->max_ctx, 64);
   h->stage_q = base + stage_q_off;
   h->stage_qidx = base + stage_qi_off;
@@ -430,7 +437,7 @@ rtp_status rtp_decode_step(rtp_handle* h, int layer, const rtp_layer_io* io, voi
   if (st != RTP_OK) return st;
   DeviceGuard guard(h->device);
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  st = enqueue_layer(h, a, s);
+  st = enqueue_layer(h, a, s, io->top_k);
   if (st != RTP_OK) return st;
   h->last_valid = true;
   h->last_stream = s;

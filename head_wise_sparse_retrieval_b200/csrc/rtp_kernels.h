@@ -31,6 +31,12 @@ struct Workspace {
   int ld;                         // per-slot stride of scores / sel_idx: max_ctx rounded up to 64
 };
 
+// Selection-only arguments (kept apart from LayerArgs, which the attention launches share).
+struct SelectArgs {
+  int top_k;                      // > 0: b* by token count (fixed top-k) instead of mass
+  unsigned* hist_cnt;             // [kHistCopies][slots][256] tokens per bin (top-k only)
+};
+
 struct LayerArgs {
   const __nv_bfloat16* q;         // [B][Hq][128]
   const __half* q_idx;            // [B][Hkv][16]
@@ -50,8 +56,8 @@ struct LayerArgs {
 // Kernel entry points (defined in select_kernels.cu / attend_kernel.cu).
 // Cooperative launches. _onchip: every CTA's range fits in shared memory (no spill code);
 // _spill: longer ranges keep the rest of their scores and bins in the global workspace.
-__global__ void select_kernel_onchip(const LayerArgs a, const Workspace w);
-__global__ void select_kernel_spill(const LayerArgs a, const Workspace w);
+__global__ void select_kernel_onchip(const LayerArgs a, const Workspace w, const SelectArgs x);
+__global__ void select_kernel_spill(const LayerArgs a, const Workspace w, const SelectArgs x);
 __global__ void attend_kernel(const LayerArgs a, const Workspace w);
 __global__ void merge_kernel(const LayerArgs a, const Workspace w);
 

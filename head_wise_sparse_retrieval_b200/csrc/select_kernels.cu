@@ -202,7 +202,8 @@ size_t select_smem_bytes(int slots) {
 }
 
 template <bool kFits>
-__device__ __forceinline__ void select_body(const LayerArgs& a, const Workspace& w) {
+__device__ __forceinline__ void select_body(const LayerArgs& a, const Workspace& w,
+                                            const SelectArgs& x) {
   extern __shared__ __align__(16) unsigned char dsm[];
   __shared__ uint32_t wlo[kWarpsSel][kBins];   // per-warp fixed-point masses, bits 0..19
   __shared__ uint32_t whi[kWarpsSel][kBins];   // bits 20..40
@@ -225,8 +226,11 @@ __device__ __forceinline__ void select_body(const LayerArgs& a, const Workspace&
   pdl_launch_dependents();
 
   slot_offsets(a, S, soff, w.status, blockIdx.x == 0);
-  if (blockIdx.x == 0)  // phase 2 accumulates into these
+  if (blockIdx.x == 0) {  // phase 2 accumulates into these
     for (int i = tid; i < kHistCopies * S * kBins; i += kSelThreads) w.hist[i] = 0ull;
+    if (x.top_k > 0)
+      for (int i = tid; i < kHistCopies * S * kBins; i += kSelThreads) x.hist_cnt[i] = 0u;
+  }
 
   const long long T = soff[S];
   const long long P = min((long long)gridDim.x, T);
@@ -350,6 +354,8 @@ __device__ __forceinline__ void select_body(const LayerArgs& a, const Workspace&
         if (v) atomicAdd(w.hist + ((size_t)copy * S + s) * kBins + tid, v);
         __syncthreads();  // the per-warp words are read before the next chunk clears them
       }
+      if (x.top_k > 0 && cnt[tid])  // fixed top-k: the slot's token count per bin
+        atomicAdd(x.hist_cnt + ((size_t)copy * S + s) * kBins + tid, cnt[tid]);
       // tokens of this CTA in bins >= tid, stored bin-major so that phase 3 reads one column
       const unsigned ge = block_suffix_sum<unsigned>(cnt[tid], reinterpret_cast<unsigned*>(redi));
       w.cta_ge[((size_t)s * kBins + tid) * gridDim.x + blockIdx.x] = ge;
@@ -382,8 +388,17 @@ __device__ __forceinline__ void select_body(const LayerArgs& a, const Workspace&
       const unsigned long long total = red64[0];
       const double target = (double)a.top_p * (double)total;
       const unsigned long long above = sfx - hv;  // mass of the bins above tid
-      if ((double)sfx >= target && (tid == kBins - 1 || !((double)above >= target)))
+      if (x.top_k > 0) {
+        // fixed top-k: the highest bin whose suffix count reaches k (none: every token)
+        unsigned hc = 0u;
+#pragma unroll
+        for (int k = 0; k < kHistCopies; ++k) hc += __ldcg(x.hist_cnt + ((size_t)k * S + s) * kBins + tid);
+        const unsigned cs = block_suffix_sum<unsigned>(hc, reinterpret_cast<unsigned*>(redi));
+        const unsigned kk = (unsigned)x.top_k;
+        if (cs >= kk && (tid == kBins - 1 || cs - hc < kk)) bstar_s = tid;
+      } else if ((double)sfx >= target && (tid == kBins - 1 || !((double)above >= target))) {
         bstar_s = tid;  // the highest bin whose suffix mass reaches p * C_0 (one thread)
+      }
       __syncthreads();
       const int bs = bstar_s;
       if (first && tid == 0) w.mass_total[s] = total;
@@ -432,13 +447,15 @@ __device__ __forceinline__ void select_body(const LayerArgs& a, const Workspace&
 }
 
 __global__ void __launch_bounds__(kSelThreads, 2) select_kernel_onchip(const LayerArgs a,
-                                                                       const Workspace w) {
-  select_body<true>(a, w);
+                                                                       const Workspace w,
+                                                                       const SelectArgs x) {
+  select_body<true>(a, w, x);
 }
 
 __global__ void __launch_bounds__(kSelThreads, 2) select_kernel_spill(const LayerArgs a,
-                                                                      const Workspace w) {
-  select_body<false>(a, w);
+                                                                      const Workspace w,
+                                                                      const SelectArgs x) {
+  select_body<false>(a, w, x);
 }
 
 }  // namespace rtp

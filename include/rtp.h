@@ -118,14 +118,18 @@ typedef struct {
     float *out;              /* fp32 [B][Hq][D], device: attention output                        */
     int32_t *sel_count;      /* optional [B][Hkv], device: receives |S| for retrieval heads and
                                 |T| for local heads; NULL to skip                                */
+    int32_t top_k;           /* 0: top-p selection. k > 0: fixed top-k through the same 256-bin
+                                histogram (the pages' top-k / top-p comparison): every bin from
+                                the top down until the bins hold >= k tokens, all N_b tokens
+                                when k >= N_b; top_p is then ignored.                           */
 } rtp_layer_io;
 
 /* Enqueues one layer of the decode step on `stream` (two kernels when the layer has retrieval
  * heads: the selection, then the attention of every head). Asynchronous: no host synchronisation,
  * no allocation, capturable in a CUDA graph (the mask is read on the host at call time and the
  * launch shapes depend only on cfg and the mask). Errors (nothing enqueued): RTP_ERR_INVALID_ARG
- * for a NULL handle / io / required pointer, a misaligned device pointer, top_p outside (0, 1]
- * or layer outside [0, num_layers); RTP_ERR_CUDA if a launch fails. Problems only the device
+ * for a NULL handle / io / required pointer, a misaligned device pointer, top_k < 0, top_p
+ * outside (0, 1] when top_k is 0, or layer outside [0, num_layers); RTP_ERR_CUDA if a launch fails. Problems only the device
  * can see (seq_lens) are reported through rtp_get_device_status. */
 RTP_API rtp_status rtp_decode_step(rtp_handle *h, int layer, const rtp_layer_io *io, void *stream);
 

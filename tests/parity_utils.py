@@ -43,7 +43,8 @@ class HeadOracle:
 
 
 def oracle_head(li: W.LayerInputs, b: int, kvh: int, is_ret: bool, top_p: float, G: int,
-                window: int = 8192, sinks: int = 4, dense: bool = False) -> HeadOracle:
+                window: int = 8192, sinks: int = 4, dense: bool = False,
+                top_k: int = 0) -> HeadOracle:
     """The oracle's result for one (b, KV head), from host copies of only what it reads."""
     N = int(li.seq_lens[b].item())
     q = u16(li.q[b, kvh * G:(kvh + 1) * G])
@@ -52,7 +53,10 @@ def oracle_head(li: W.LayerInputs, b: int, kvh: int, is_ret: bool, top_p: float,
         hs, s = None, None
     elif is_ret:
         s = oracle.indexer_scores(u16(li.q_idx[b, kvh]), u16(li.k_idx[b, kvh, :N]), 0.25)
-        hs = oracle.hist_topp(s, float(np.float32(top_p)))
+        if top_k > 0:
+            hs = oracle.hist_topk(s, top_k)
+        else:
+            hs = oracle.hist_topp(s, float(np.float32(top_p)))
         sel = hs.sel
     else:
         sel = oracle.window_sink_set(N, window, sinks)
@@ -108,6 +112,37 @@ def check_selection(gpu_sel: np.ndarray, gpu_bstar: int, ho: HeadOracle, top_p: 
                            gpu_bstar)
 
 
+def check_selection_topk(gpu_sel: np.ndarray, gpu_bstar: int, ho: HeadOracle,
+                         k: int) -> SelectionReport:
+    """Fixed top-k: b* is the bin of the k-th highest score, so a different b* is accepted only
+    when some token lies within EDGE_TOL of a bin edge between the two (its fp32 bin can
+    differ, which moves the counts)."""
+    s, hs = ho.scores, ho.hist
+    s_max = s.max()
+    ambiguous = False
+    ref_bstar = hs.bstar
+    if gpu_bstar != hs.bstar:
+        lo_b, hi_b = sorted((gpu_bstar, hs.bstar))
+        edges = (s_max - 16.0) + np.arange(lo_b, hi_b + 2) / 16.0
+        near = np.abs(s[:, None] - edges[None, :]).min() < EDGE_TOL
+        assert near, f"threshold bin differs: gpu {gpu_bstar}, oracle {hs.bstar}, k={k}"
+        ambiguous = True
+        ref_bstar = gpu_bstar
+    ref = set(np.nonzero(hs.bins >= ref_bstar)[0].tolist())
+    got = set(gpu_sel.tolist())
+    diff = np.array(sorted(ref ^ got), dtype=np.int64)
+    if diff.size:
+        x = (s[diff] - (s_max - 16.0)) * 16.0
+        dist = np.abs(x - np.round(x)) / 16.0
+        bad = diff[dist >= EDGE_TOL]
+        assert bad.size == 0, f"{bad.size} selection differences away from bin edges"
+    assert np.all(np.diff(gpu_sel) > 0), "selection must be strictly ascending"
+    assert len(got) >= min(k, s.size)
+    n_exact = oracle.exact_topk(s, k).size
+    return SelectionReport(len(ref), len(got), n_exact, int(diff.size), ambiguous, hs.bstar,
+                           gpu_bstar)
+
+
 def check_output(gpu: np.ndarray, ref: np.ndarray, what: str = ""):
     err = np.abs(gpu.astype(np.float64) - ref)
     assert np.isfinite(gpu).all(), f"{what}: non-finite output"
@@ -121,7 +156,7 @@ def make_handle(plan: W.Plan, **cfg_overrides) -> rtp.Handle:
 
 
 def run_layer(h: rtp.Handle, plan: W.Plan, li: W.LayerInputs, layer: int, top_p=None,
-              dense=False):
+              dense=False, top_k: int = 0):
     B, Hq, Hkv = plan.batch, plan.num_q_heads, plan.num_kv_heads
     out = torch.full((B, Hq, 128), float("nan"), dtype=torch.float32, device=li.q.device)
     cnt = torch.full((B, Hkv), -1, dtype=torch.int32, device=li.q.device)
@@ -130,7 +165,7 @@ def run_layer(h: rtp.Handle, plan: W.Plan, li: W.LayerInputs, layer: int, top_p=
         h.dense_decode(L, out)
     else:
         h.decode_step(layer, L, plan.retrieval[layer], plan.top_p if top_p is None else top_p,
-                      out, cnt)
+                      out, cnt, top_k=top_k)
     torch.cuda.synchronize()
     return out, cnt
 
@@ -143,10 +178,10 @@ class LayerReport:
 
 
 def check_layer(h: rtp.Handle, plan: W.Plan, li: W.LayerInputs, layer: int, top_p=None,
-                heads=None, exact=True) -> LayerReport:
+                heads=None, exact=True, top_k: int = 0) -> LayerReport:
     """Run one layer on the GPU and compare every (or the given) head with the oracle."""
     p = plan.top_p if top_p is None else top_p
-    out, cnt = run_layer(h, plan, li, layer, p)
+    out, cnt = run_layer(h, plan, li, layer, p, top_k=top_k)
     assert h.device_status() == 0
     G = plan.group
     rep = LayerReport()
@@ -157,12 +192,15 @@ def check_layer(h: rtp.Handle, plan: W.Plan, li: W.LayerInputs, layer: int, top_
     cnt_h = cnt.cpu().numpy()
     for b, kvh in todo:
         is_ret = bool(plan.retrieval[layer, kvh])
-        ho = oracle_head(li, b, kvh, is_ret, p, G, plan.window, plan.sinks)
+        ho = oracle_head(li, b, kvh, is_ret, p, G, plan.window, plan.sinks, top_k=top_k)
         info = {"b": b, "kvh": kvh, "ret": is_ret, "n_sel": int(ho.sel.size)}
         if is_ret:
             gsel = h.selection(b, kvh)
             gb, _ = h.threshold(b, kvh)
-            sr = check_selection(gsel, gb, ho, p, exact=exact)
+            if top_k > 0:
+                sr = check_selection_topk(gsel, gb, ho, top_k)
+            else:
+                sr = check_selection(gsel, gb, ho, p, exact=exact)
             info["sel"] = sr
             assert cnt_h[b, kvh] == gsel.size
             if sr.edge_tokens == 0 and not sr.ambiguous:

@@ -21,10 +21,10 @@ def _needs_gpu():
     rtp.load()
 
 
-def _run(plan, layer=0, top_p=None, heads=None, poison=False, exact=True, **cfg):
+def _run(plan, layer=0, top_p=None, heads=None, poison=False, exact=True, top_k=0, **cfg):
     li = W.make_layer(plan, layer, DEV, poison_tail=poison)
     with make_handle(plan, **cfg) as h:
-        rep = check_layer(h, plan, li, layer, top_p, heads, exact=exact)
+        rep = check_layer(h, plan, li, layer, top_p, heads, exact=exact, top_k=top_k)
     return rep
 
 
@@ -90,6 +90,28 @@ def test_top_p_values(top_p):
     rep = _run(p, top_p=top_p)
     if top_p == 1.0:
         assert all(h["sel"].n_gpu == 30000 for h in rep.heads)
+
+
+@pytest.mark.parametrize("query", ["diffuse", "flat", "conc"])
+@pytest.mark.parametrize("k", [1, 2048, 4096, 16384])
+def test_fixed_top_k(query, k):
+    """Fixed top-k through the histogram (the pages' top-2k / 4k / 16k): every bin from the top
+    until the bins hold k tokens."""
+    p = W.plan("one_layer", query=query)
+    rep = _run(p, top_k=k)
+    r = rep.heads[0]["sel"]
+    assert r.n_gpu >= k and r.n_exact == k
+
+
+def test_fixed_top_k_ragged_and_beyond_n():
+    seq = [100, 5000, 40000, 3]
+    kinds = [[W.KIND_DIFFUSE, W.KIND_FLAT]] * 4
+    p = W.custom(batch=4, num_q_heads=16, num_kv_heads=2, seq_lens=seq, max_ctx=40000,
+                 retrieval=[1, 1], kinds=kinds, seed=31)
+    rep = _run(p, top_k=4096, poison=True)
+    for h in rep.heads:
+        n = seq[h["b"]]
+        assert h["sel"].n_gpu == n if n <= 4096 else h["sel"].n_gpu >= 4096
 
 
 def test_small_window_and_no_sinks():
@@ -228,6 +250,19 @@ def test_bad_seq_len_is_reported_not_faulted():
         assert code & rtp.DEV_BAD_SEQLEN
         assert h.device_status() == 0  # reading clears it
     assert torch.isfinite(out[0]).all()
+
+
+def test_negative_top_k_is_rejected():
+    p = W.plan("tiny")
+    li = W.make_layer(p, 0, DEV)
+    with make_handle(p) as h:
+        out = torch.empty((1, 8, 128), dtype=torch.float32, device=DEV)
+        with pytest.raises(rtp.RtpError) as e:
+            h.decode_step(0, rtp.layer_from(li), [1], 0.9, out, top_k=-1)
+        assert e.value.status == rtp.RTP_ERR_INVALID_ARG
+        h.decode_step(0, rtp.layer_from(li), [1], 0.0, out, top_k=5)  # top_p ignored
+        torch.cuda.synchronize()
+        assert h.selection(0, 0).size >= 5
 
 
 def test_host_side_argument_errors():
