@@ -197,7 +197,11 @@ __global__ void __launch_bounds__(kAttendThreads, kAttendCtasPerSm) attend_kerne
   int* sSeq = reinterpret_cast<int*>(smem + SmemLayout::seq_off(nheads));
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  pdl_wait();
+  // Without retrieval heads nothing here depends on the launch before (the previous layer's
+  // merge, which reads the partials this kernel writes). When the caller vouches that the
+  // inputs are ready, the wait moves to just before the first write.
+  const bool early = a.early && (a.nret == 0 || a.dense);
+  if (!early) pdl_wait();
 
   // ---- the layer's heads and their token-set lengths --------------------------------------
   for (int hd = tid; hd < nheads; hd += kAttendThreads) {
@@ -400,6 +404,7 @@ __global__ void __launch_bounds__(kAttendThreads, kAttendCtasPerSm) attend_kerne
     }
     kseg += nt;
 
+    if (early) pdl_wait();  // the partials below may still be read by the previous merge
     // ---- end of this head's piece: merge the warps ----------------------------------------
     // (m, l) per warp and head through shared memory; each warp rescales its O in registers
     // to the common max, then the warps add O into one buffer in a fixed order.

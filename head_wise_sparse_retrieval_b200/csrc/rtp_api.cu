@@ -202,6 +202,7 @@ LayerArgs make_args(const rtp_handle* h, const rtp_layer_io* io) {
   a.window = h->cfg.window;
   a.sinks = h->cfg.sinks;
   a.top_p = io->top_p;
+  a.early = io->inputs_ready ? 1 : 0;
   a.idx_scale = h->cfg.idx_scale;
   a.attn_scale_log2 = (float)((double)h->cfg.attn_scale * 1.4426950408889634);
   a.bin_scale = (float)((double)kBins / (double)h->cfg.idx_range);
@@ -503,6 +504,7 @@ rtp_status rtp_decode_step_host(rtp_handle* h, int num_layers, const void* q_hos
       io.retrieval_mask = masks + (size_t)l * c.num_kv_heads;
       io.top_p = top_p;
       io.out = h->stage_out + (size_t)l * q_layer;
+      io.inputs_ready = 1;  // staged before the first launch; the caches do not change
       rtp_status st = rtp_decode_step(h, l, &io, st_stream);
       if (st != RTP_OK) return st;
     }

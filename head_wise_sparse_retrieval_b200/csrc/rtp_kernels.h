@@ -51,6 +51,8 @@ struct LayerArgs {
   float top_p, idx_scale, attn_scale_log2, bin_scale;
   short ret_kvh[kMaxKvHeads];     // KV head of retrieval index j (j < nret)
   short slot_of_kvh[kMaxKvHeads]; // retrieval index j of KV head kvh, or -1 for a local head
+  int early;                      // the caller vouches the inputs are complete before the
+                                  // preceding launch ends: kernels may read them before waiting
 };
 
 // Kernel entry points (defined in select_kernels.cu / attend_kernel.cu).

@@ -222,7 +222,11 @@ __device__ __forceinline__ void select_body(const LayerArgs& a, const Workspace&
   long long* soff = reinterpret_cast<long long*>(dsm + (size_t)kScoreCap * 5);
   if (tid == 0) aborted = 0;
 
-  pdl_wait();
+  // Nothing this kernel writes is read by the launch before it (the previous layer's merge),
+  // and the selection lists it overwrites were consumed before that merge began. So when the
+  // caller vouches that the inputs are ready (a.early), the wait moves to the kernel's end:
+  // it still finishes only after its predecessor, which the next launch relies on.
+  if (!a.early) pdl_wait();
   pdl_launch_dependents();
 
   slot_offsets(a, S, soff, w.status, blockIdx.x == 0);
@@ -444,6 +448,7 @@ __device__ __forceinline__ void select_body(const LayerArgs& a, const Workspace&
       __syncthreads();
     }
   }
+  if (a.early) pdl_wait();
 }
 
 __global__ void __launch_bounds__(kSelThreads, 2) select_kernel_onchip(const LayerArgs a,

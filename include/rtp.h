@@ -122,6 +122,14 @@ typedef struct {
                                 histogram (the pages' top-k / top-p comparison): every bin from
                                 the top down until the bins hold >= k tokens, all N_b tokens
                                 when k >= N_b; top_p is then ignored.                           */
+    int32_t inputs_ready;    /* 0 (safe default): the layer's kernels wait for the preceding
+                                launch on the stream before reading anything. Nonzero: the caller
+                                vouches that q, q_idx, seq_lens and the caches are complete before
+                                that launch ends (e.g. layer after layer of one step with every
+                                input already resident), so the selection scores and the
+                                attention of a layer without retrieval heads stream their inputs
+                                while the previous launch drains; they still wait before
+                                writing anything the previous layer may read.                   */
 } rtp_layer_io;
 
 /* Enqueues one layer of the decode step on `stream` (two kernels when the layer has retrieval

@@ -239,6 +239,32 @@ def test_host_buffer_entry_matches_device_entry():
             assert torch.equal(out[l], dev_out3[l].cpu())
 
 
+def test_inputs_ready_chaining_matches_strict_ordering():
+    """Layers launched back to back with inputs_ready (selection scoring and local-only
+    attention start before the previous launch finishes) give bit-identical outputs and
+    selections to the strictly ordered launches."""
+    p = W.plan("long_context", num_layers=6, ctx=30000)
+    lis = [W.make_layer(p, l, DEV) for l in range(6)]
+    B, Hq, Hkv = p.batch, p.num_q_heads, p.num_kv_heads
+    with make_handle(p) as h:
+        res = {}
+        for ready in (False, True):
+            outs = [torch.full((B, Hq, 128), float("nan"), device=DEV) for _ in lis]
+            cnts = [torch.full((B, Hkv), -1, dtype=torch.int32, device=DEV) for _ in lis]
+            for rep in range(3):
+                for l, li in enumerate(lis):
+                    h.decode_step(l, rtp.layer_from(li), p.retrieval[l], p.top_p, outs[l],
+                                  cnts[l], inputs_ready=ready)
+            torch.cuda.synchronize()
+            assert h.device_status() == 0
+            res[ready] = ([o.cpu() for o in outs], [c.cpu() for c in cnts])
+    assert any(p.retrieval[l].any() for l in range(6)) and not all(p.retrieval[l].any()
+                                                                    for l in range(6))
+    for l in range(6):
+        assert torch.equal(res[True][0][l], res[False][0][l])
+        assert torch.equal(res[True][1][l], res[False][1][l])
+
+
 def test_bad_seq_len_is_reported_not_faulted():
     p = W.custom(batch=2, num_q_heads=8, num_kv_heads=1, seq_lens=[100, 50], max_ctx=128,
                  retrieval=[1], kinds=[[W.KIND_CONC]] * 2, n_needles=[[2]] * 2, seed=14)
