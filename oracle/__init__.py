@@ -54,6 +54,8 @@ def lib():
         L.orc_hist_topp.argtypes = [_dp, ctypes.c_int64, ctypes.c_double, ctypes.c_double,
                                     ctypes.c_int, _ip, _dp, _dp, _ip, _i64p, _i64p]
         L.orc_exact_topp.argtypes = [_dp, ctypes.c_int64, ctypes.c_double, _i64p, _i64p]
+        L.orc_indexer_project.argtypes = [_u16p, _u16p, _u16p, _u16p, ctypes.c_int, ctypes.c_int,
+                                          ctypes.c_int, ctypes.c_int, ctypes.c_int, _dp, _dp]
         L.orc_hist_topk.argtypes = [_dp, ctypes.c_int64, ctypes.c_int64, ctypes.c_double,
                                     ctypes.c_int, _ip, _i64p, _i64p, _ip, _i64p, _i64p]
         L.orc_exact_topk.argtypes = [_dp, ctypes.c_int64, ctypes.c_int64, _i64p, _i64p]
@@ -108,6 +110,22 @@ def indexer_scores(q_idx, k_idx, scale: float = 0.25) -> np.ndarray:
     _check(lib().orc_indexer_scores(_ptr(q, ctypes.c_uint16), _ptr(k, ctypes.c_uint16), n, r,
                                     scale, _ptr(s, ctypes.c_double)), "indexer_scores")
     return s
+
+
+def indexer_project(q_pre, k_pre, w_q, w_k):
+    """(q_idx, k_idx) fp64 [B, Hkv, r] from bf16 bits q_pre [B, Hq, D], k_pre [B, Hkv, D],
+    w_q [Hkv, r, G*D], w_k [Hkv, r, D]."""
+    q_pre, k_pre, w_q, w_k = _u16(q_pre), _u16(k_pre), _u16(w_q), _u16(w_k)
+    B, Hq, D = q_pre.shape
+    Hkv, r, GD = w_q.shape
+    assert k_pre.shape == (B, Hkv, D) and w_k.shape == (Hkv, r, D) and GD == (Hq // Hkv) * D
+    qi = np.empty((B, Hkv, r), np.float64)
+    ki = np.empty((B, Hkv, r), np.float64)
+    _check(lib().orc_indexer_project(_ptr(q_pre, ctypes.c_uint16), _ptr(k_pre, ctypes.c_uint16),
+                                     _ptr(w_q, ctypes.c_uint16), _ptr(w_k, ctypes.c_uint16), B,
+                                     Hq, Hkv, D, r, _ptr(qi, ctypes.c_double),
+                                     _ptr(ki, ctypes.c_double)), "indexer_project")
+    return qi, ki
 
 
 @dataclass
@@ -250,7 +268,8 @@ def max_threads() -> int:
 
 __all__ = [
     "MODE_HIST", "MODE_EXACT", "MODE_DENSE", "bf16_to_f64", "f16_to_f64", "indexer_scores",
-    "hist_topp", "HistSelection", "exact_topp", "hist_topk", "HistTopK", "exact_topk",
+    "indexer_project", "hist_topp", "HistSelection", "exact_topp", "hist_topk", "HistTopK",
+    "exact_topk",
     "window_sink_set", "sparse_attention",
     "decode_layer", "max_threads",
 ]

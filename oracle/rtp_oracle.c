@@ -22,8 +22,9 @@
  *
  * Readings taken where the pages are silent (each is also listed in the design notes):
  *   - the indexer score is scaled by 1/sqrt(r) (r = 16 -> 0.25) before anything else;
- *   - the query-side projection W^Q q^pre is done by the caller: this oracle receives q_idx
- *     and the cached 16-d keys W^K k^pre directly;
+ *   - the decode step receives q_idx = W^Q q^pre and the cached 16-d keys W^K k^pre; the
+ *     projections themselves (orc_indexer_project) map a KV head's group of G pre-RoPE query
+ *     heads, concatenated head-major (G * D values), and its pre-RoPE key (D values) to r dims;
  *   - the attention mass of token n is w_n = exp(s_n - s_max) (softmax up to the common
  *     normaliser, which cancels in the "reaches p" comparison);
  *   - the 256 bins have equal width over [s_max - range, s_max] (range = 16) of the scaled
@@ -93,6 +94,45 @@ int orc_indexer_scores(const uint16_t *q_idx, const uint16_t *k_idx, int64_t n_t
         for (int i = 0; i < r; i++)
             acc += orc_f16_to_f64(q_idx[i]) * orc_f16_to_f64(k_idx[n * r + i]);
         s[n] = scale * acc;
+    }
+    return ORC_OK;
+}
+
+/* ---- indexer production [P1 自适应稀疏注意力: W^Q_h q^pre, W^K_h k^pre, before RoPE] ---- */
+
+/*
+ * For sequence b and KV head h (G = Hq / Hkv query heads per KV head, D = head_dim):
+ *   q_idx[b][h][i] = sum_{j < G*D} wq[h][i][j] * q_pre[b][h*G + j/D][j%D]
+ *   k_idx[b][h][i] = sum_{d < D}   wk[h][i][d] * k_pre[b][h][d]
+ * over the bf16 inputs in fp64; the caller rounds to the 16-bit storage format.
+ * Layouts: q_pre [B][Hq][D], k_pre [B][Hkv][D], wq [Hkv][r][G*D], wk [Hkv][r][D] (bf16 bits);
+ * q_idx, k_idx [B][Hkv][r] fp64.
+ */
+int orc_indexer_project(const uint16_t *q_pre, const uint16_t *k_pre, const uint16_t *wq,
+                        const uint16_t *wk, int B, int Hq, int Hkv, int D, int r, double *q_idx,
+                        double *k_idx)
+{
+    if (!q_pre || !k_pre || !wq || !wk || !q_idx || !k_idx || B <= 0 || Hkv <= 0 || D <= 0 ||
+        r <= 0 || Hq % Hkv != 0)
+        return ORC_ERR_ARG;
+    const int G = Hq / Hkv;
+    const int64_t GD = (int64_t)G * D;
+    for (int b = 0; b < B; b++) {
+        for (int h = 0; h < Hkv; h++) {
+            const uint16_t *qg = q_pre + ((int64_t)b * Hq + (int64_t)h * G) * D;
+            const uint16_t *kh = k_pre + ((int64_t)b * Hkv + h) * D;
+            for (int i = 0; i < r; i++) {
+                const uint16_t *wqr = wq + ((int64_t)h * r + i) * GD;
+                const uint16_t *wkr = wk + ((int64_t)h * r + i) * D;
+                double aq = 0.0, ak = 0.0;
+                for (int64_t j = 0; j < GD; j++)
+                    aq += orc_bf16_to_f64(wqr[j]) * orc_bf16_to_f64(qg[j]);
+                for (int d = 0; d < D; d++)
+                    ak += orc_bf16_to_f64(wkr[d]) * orc_bf16_to_f64(kh[d]);
+                q_idx[((int64_t)b * Hkv + h) * r + i] = aq;
+                k_idx[((int64_t)b * Hkv + h) * r + i] = ak;
+            }
+        }
     }
     return ORC_OK;
 }

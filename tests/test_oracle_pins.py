@@ -209,6 +209,57 @@ def test_hist_brute_force_tiny(orc):
 
 # ---- window + sinks --------------------------------------------------------------------
 
+# ---- indexer production (W^Q q^pre, W^K k^pre) ------------------------------------------
+
+def _bf16_round(x):
+    return torch.as_tensor(np.asarray(x, np.float32)).to(torch.bfloat16).float().numpy()
+
+
+def test_indexer_project_selector_weights(orc):
+    """One-hot rows of W pick single input coordinates: the outputs are those coordinates
+    exactly, which pins the head-major concatenation of the group's queries and the layouts."""
+    B, Hq, Hkv, D, r = 2, 8, 2, 128, 16
+    G = Hq // Hkv
+    rng = np.random.default_rng(5)
+    q = _bf16_round(rng.normal(0, 1, (B, Hq, D)))
+    k = _bf16_round(rng.normal(0, 1, (B, Hkv, D)))
+    wq = np.zeros((Hkv, r, G * D), np.float32)
+    wk = np.zeros((Hkv, r, D), np.float32)
+    pick_q = rng.integers(0, G * D, (Hkv, r))
+    pick_k = rng.integers(0, D, (Hkv, r))
+    for h in range(Hkv):
+        for i in range(r):
+            wq[h, i, pick_q[h, i]] = 1.0
+            wk[h, i, pick_k[h, i]] = -2.0
+    qi, ki = orc.indexer_project(_bf16_bits(q), _bf16_bits(k), _bf16_bits(wq), _bf16_bits(wk))
+    for b in range(B):
+        for h in range(Hkv):
+            for i in range(r):
+                j = pick_q[h, i]
+                assert qi[b, h, i] == q[b, h * G + j // D, j % D]
+                assert ki[b, h, i] == -2.0 * k[b, h, pick_k[h, i]]
+
+
+def test_indexer_project_matches_einsum(orc):
+    B, Hq, Hkv, D, r = 3, 16, 4, 128, 16
+    G = Hq // Hkv
+    rng = np.random.default_rng(6)
+    q = _bf16_round(rng.normal(0, 1, (B, Hq, D)))
+    k = _bf16_round(rng.normal(0, 1, (B, Hkv, D)))
+    wq = _bf16_round(rng.normal(0, 0.05, (Hkv, r, G * D)))
+    wk = _bf16_round(rng.normal(0, 0.1, (Hkv, r, D)))
+    qi, ki = orc.indexer_project(_bf16_bits(q), _bf16_bits(k), _bf16_bits(wq), _bf16_bits(wk))
+    ref_q = np.einsum("hij,bhj->bhi", wq.astype(np.float64),
+                      q.astype(np.float64).reshape(B, Hkv, G * D))
+    ref_k = np.einsum("hid,bhd->bhi", wk.astype(np.float64), k.astype(np.float64))
+    assert np.allclose(qi, ref_q, rtol=1e-12, atol=1e-12)
+    assert np.allclose(ki, ref_k, rtol=1e-12, atol=1e-12)
+    # linear in the weights
+    qi2, ki2 = orc.indexer_project(_bf16_bits(q), _bf16_bits(k), _bf16_bits(2 * wq),
+                                   _bf16_bits(-wk))
+    assert np.allclose(qi2, 2 * qi, rtol=1e-14) and np.allclose(ki2, -ki, rtol=1e-14)
+
+
 # ---- fixed top-k through the histogram --------------------------------------------------
 
 def test_hist_topk_golden_counts(orc):
