@@ -448,6 +448,39 @@ def main():
     # so each layer's scoring / local attention streams while the previous launch drains
     chained = time_variant(plan.top_p, 0, ready=True)
 
+    # indexer production of one layer (q_idx and the new k_idx row of every KV head), timed as a
+    # CUDA graph of 100 calls; W is random (no trained weights), the row goes to a scratch cache
+    G = Hq // Hkv
+    gen = torch.Generator(device=dev).manual_seed(99)
+    q_pre = torch.randn(B, Hq, 128, generator=gen, device=dev).to(torch.bfloat16)
+    k_pre = torch.randn(B, Hkv, 128, generator=gen, device=dev).to(torch.bfloat16)
+    w_q = (0.03 * torch.randn(Hkv, 16, G * 128, generator=gen, device=dev)).to(torch.bfloat16)
+    w_k = (0.1 * torch.randn(Hkv, 16, 128, generator=gen, device=dev)).to(torch.bfloat16)
+    qi_s = torch.empty(B, Hkv, 16, dtype=torch.float16, device=dev)
+    ki_s = torch.empty(B, Hkv, plan.max_ctx, 16, dtype=torch.float16, device=dev)
+    seq_d = layers[0].seq_lens
+    with torch.cuda.stream(stream):
+        h.indexer_append(q_pre, k_pre, w_q, w_k, seq_d, qi_s, ki_s, stream=stream)
+    torch.cuda.synchronize()
+    gi = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(gi, stream=stream):
+        for _ in range(100):
+            h.indexer_append(q_pre, k_pre, w_q, w_k, seq_d, qi_s, ki_s, stream=stream)
+    with torch.cuda.stream(stream):
+        gi.replay()
+        i0 = torch.cuda.Event(enable_timing=True)
+        i1 = torch.cuda.Event(enable_timing=True)
+        i0.record(stream)
+        gi.replay()
+        i1.record(stream)
+    torch.cuda.synchronize()
+    ius = i0.elapsed_time(i1) * 1e3 / 100
+    ibytes = 2 * (w_q.numel() + w_k.numel() + q_pre.numel() + k_pre.numel() + 2 * B * Hkv * 16)
+    indexer = {"us_per_call": ius, "bytes_per_call": ibytes,
+               "effective_gbs": ibytes / (ius * 1e-6) / 1e9,
+               "shape": {"batch": B, "q_heads": Hq, "kv_heads": Hkv, "r": 16}}
+    del gi, ki_s
+
     # dense decode on the same caches (the speedup denominator)
     dense = None
     if not args.no_dense:
@@ -547,6 +580,7 @@ def main():
         "p_sweep": p_sweep,
         "k_sweep": k_sweep,
         "chained": chained,
+        "indexer_append": indexer,
         "dense": dense,
         "e2e": e2e,
         "cpu_baseline": cpu,

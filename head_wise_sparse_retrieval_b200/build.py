@@ -7,7 +7,8 @@ PKG = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 LIB = os.path.join(PKG, "librtp.so")
-SOURCES = ["rtp_api.cu", "select_kernels.cu", "attend_kernel.cu", "noalloc.cu"]
+SOURCES = ["rtp_api.cu", "select_kernels.cu", "attend_kernel.cu", "noalloc.cu",
+           "indexer_kernel.cu"]
 HEADERS = ["rtp_device.cuh", "rtp_kernels.h"]
 NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")
 FLAGS = ["-gencode", "arch=compute_100a,code=sm_100a", "-O3", "-lineinfo", "-std=c++17",

@@ -447,6 +447,46 @@ rtp_status rtp_decode_step(rtp_handle* h, int layer, const rtp_layer_io* io, voi
   return ok();
 }
 
+rtp_status rtp_indexer_append(rtp_handle* h, const rtp_indexer_io* io, void* stream) {
+  if (!h) return fail(RTP_ERR_INVALID_ARG, "handle is NULL");
+  if (!io || !io->q_pre || !io->k_pre || !io->w_q || !io->w_k || !io->seq_lens || !io->q_idx ||
+      !io->k_idx)
+    return fail(RTP_ERR_INVALID_ARG, "a required pointer is NULL");
+  if (!aligned16(io->q_pre) || !aligned16(io->k_pre) || !aligned16(io->w_q) ||
+      !aligned16(io->w_k) || !aligned16(io->q_idx) || !aligned16(io->k_idx) ||
+      ((uintptr_t)io->seq_lens & 3u))
+    return fail(RTP_ERR_INVALID_ARG, "pointers must be 16-byte aligned (seq_lens 4)");
+  IndexerArgs x;
+  memset(&x, 0, sizeof x);
+  x.q_pre = static_cast<const __nv_bfloat16*>(io->q_pre);
+  x.k_pre = static_cast<const __nv_bfloat16*>(io->k_pre);
+  x.w_q = static_cast<const __nv_bfloat16*>(io->w_q);
+  x.w_k = static_cast<const __nv_bfloat16*>(io->w_k);
+  x.seq_lens = io->seq_lens;
+  x.q_idx = static_cast<__half*>(io->q_idx);
+  x.k_idx = static_cast<__half*>(io->k_idx);
+  x.status = h->ws.status;
+  x.Hq = h->cfg.num_q_heads;
+  x.Hkv = h->cfg.num_kv_heads;
+  x.G = h->G;
+  x.max_ctx = h->cfg.max_ctx;
+  for (int k = 0; k < x.Hkv; ++k)
+    if (!io->head_mask || io->head_mask[k]) x.heads[x.nsel++] = (short)k;
+  if (x.nsel == 0) return ok();
+  DeviceGuard guard(h->device);
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(h->cfg.batch * x.nsel);
+  cfg.blockDim = dim3(128);
+  cfg.stream = static_cast<cudaStream_t>(stream);
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  cudaError_t e = cudaLaunchKernelEx(&cfg, indexer_kernel, x);
+  return e == cudaSuccess ? ok() : cuda_fail(e, "indexer_kernel launch");
+}
+
 rtp_status rtp_dense_decode(rtp_handle* h, const rtp_layer_io* io, void* stream) {
   if (!h) return fail(RTP_ERR_INVALID_ARG, "handle is NULL");
   rtp_status st = check_io(h, io, false);

@@ -55,6 +55,22 @@ struct LayerArgs {
                                   // preceding launch ends: kernels may read them before waiting
 };
 
+// Indexer production at decode (indexer_kernel.cu).
+struct IndexerArgs {
+  const __nv_bfloat16* q_pre;     // [B][Hq][128]
+  const __nv_bfloat16* k_pre;     // [B][Hkv][128]
+  const __nv_bfloat16* w_q;       // [Hkv][16][G*128]
+  const __nv_bfloat16* w_k;       // [Hkv][16][128]
+  const int* seq_lens;            // [B]
+  __half* q_idx;                  // [B][Hkv][16]
+  __half* k_idx;                  // [B][Hkv][max_ctx][16], row N_b - 1 written
+  unsigned* status;
+  int Hq, Hkv, G, max_ctx;
+  int nsel;                       // KV heads produced, listed in heads[]
+  short heads[kMaxKvHeads];
+};
+__global__ void indexer_kernel(const IndexerArgs x);
+
 // Kernel entry points (defined in select_kernels.cu / attend_kernel.cu).
 // Cooperative launches. _onchip: every CTA's range fits in shared memory (no spill code);
 // _spill: longer ranges keep the rest of their scores and bins in the global workspace.

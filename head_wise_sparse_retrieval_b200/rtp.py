@@ -24,7 +24,8 @@ DEV_BAD_SEQLEN, DEV_WAIT_TIMEOUT, DEV_BAD_INDEX = 0x1, 0x2, 0x4
 EXPORTS = ("rtp_config_default", "rtp_workspace_bytes", "rtp_create", "rtp_destroy",
            "rtp_decode_step", "rtp_dense_decode", "rtp_decode_step_host", "rtp_get_selection",
            "rtp_get_threshold", "rtp_get_device_status", "rtp_status_string", "rtp_last_error",
-           "rtp_profile_enable", "rtp_profile_read", "rtp_window_attention_noalloc")
+           "rtp_profile_enable", "rtp_profile_read", "rtp_window_attention_noalloc",
+           "rtp_indexer_append")
 NOALLOC_MAX_HEADS = 64
 KERNEL_CLASSES = ("select", "attend", "merge", "reserved3")
 
@@ -50,6 +51,15 @@ class NoAllocParams(ctypes.Structure):
         ("batch", ctypes.c_int), ("num_q_heads", ctypes.c_int), ("num_kv_heads", ctypes.c_int),
         ("max_ctx", ctypes.c_int), ("window", ctypes.c_int), ("sinks", ctypes.c_int),
         ("attn_scale", ctypes.c_float), ("dense", ctypes.c_int),
+    ]
+
+
+class IndexerIO(ctypes.Structure):
+    _fields_ = [
+        ("q_pre", ctypes.c_void_p), ("k_pre", ctypes.c_void_p), ("w_q", ctypes.c_void_p),
+        ("w_k", ctypes.c_void_p), ("seq_lens", ctypes.c_void_p),
+        ("head_mask", ctypes.POINTER(ctypes.c_uint8)), ("q_idx", ctypes.c_void_p),
+        ("k_idx", ctypes.c_void_p),
     ]
 
 
@@ -97,6 +107,8 @@ def load(path: str = LIB_PATH):
     L.rtp_window_attention_noalloc.argtypes = [ctypes.POINTER(NoAllocParams), vp, vp, vp, vp,
                                                vp, vp]
     L.rtp_window_attention_noalloc.restype = ctypes.c_int
+    L.rtp_indexer_append.argtypes = [vp, ctypes.POINTER(IndexerIO), vp]
+    L.rtp_indexer_append.restype = ctypes.c_int
     L.rtp_status_string.argtypes = [i]
     L.rtp_status_string.restype = ctypes.c_char_p
     L.rtp_last_error.argtypes = []
@@ -215,6 +227,20 @@ class Handle:
             self._h, L, _ptr(q_host), _ptr(q_idx_host), _ptr(seq_lens_host), kc, vc, ki,
             m.ctypes.data_as(ctypes.POINTER(ctypes.c_uint8)), float(top_p), _ptr(out_host),
             _stream_ptr(stream)), "rtp_decode_step_host")
+
+    def indexer_append(self, q_pre, k_pre, w_q, w_k, seq_lens, q_idx, k_idx, head_mask=None,
+                       stream=None):
+        """rtp_indexer_append: q_idx and the new k_idx row from the pre-RoPE q / k."""
+        m = None
+        mp = ctypes.POINTER(ctypes.c_uint8)()
+        if head_mask is not None:
+            m = np.ascontiguousarray(np.asarray(head_mask, dtype=np.uint8))
+            assert m.shape == (self.cfg.num_kv_heads,)
+            mp = m.ctypes.data_as(ctypes.POINTER(ctypes.c_uint8))
+        io = IndexerIO(_ptr(q_pre), _ptr(k_pre), _ptr(w_q), _ptr(w_k), _ptr(seq_lens), mp,
+                       _ptr(q_idx), _ptr(k_idx))
+        _check(load().rtp_indexer_append(self._h, ctypes.byref(io), _stream_ptr(stream)),
+               "rtp_indexer_append")
 
     def selection(self, b: int, kvh: int) -> np.ndarray:
         """Ascending positions selected for (b, kvh) by the last decode_step."""

@@ -141,6 +141,30 @@ typedef struct {
  * can see (seq_lens) are reported through rtp_get_device_status. */
 RTP_API rtp_status rtp_decode_step(rtp_handle *h, int layer, const rtp_layer_io *io, void *stream);
 
+/* ---- Indexer production at decode ----------------------------------------------------
+ * [R] section 三 核心公式 / 自适应稀疏注意力: the retrieval score uses low-rank projections of
+ * the query and key taken before RoPE, s_h(m,n) = (W^Q_h q^pre_{m,h})^T (W^K_h k^pre_{n,h}).
+ * rtp_indexer_append produces, for the current token of every sequence b and every selected
+ * KV head h, the indexer query of rtp_decode_step and the new indexer-key cache row:
+ *   q_idx[b][h][i]         = fp16( sum_{j < G*D} w_q[h][i][j] * q_pre[b][h*G + j/D][j%D] )
+ *   k_idx[b][h][N_b-1][i]  = fp16( sum_{d < D}   w_k[h][i][d] * k_pre[b][h][d] )
+ * (the G query heads of the KV head's group concatenated head-major; fp32 accumulation,
+ * rounded to nearest fp16 once). All pointers are device memory, 16-byte aligned except
+ * seq_lens (4). Errors: RTP_ERR_INVALID_ARG for NULL / misaligned pointers; a seq_lens entry
+ * outside [1, max_ctx] is clamped and reported in the device status word. */
+typedef struct {
+    const void *q_pre;       /* bf16 [B][Hq][D]: pre-RoPE queries of the current token         */
+    const void *k_pre;       /* bf16 [B][Hkv][D]: pre-RoPE key of the current token            */
+    const void *w_q;         /* bf16 [Hkv][r][G*D]                                             */
+    const void *w_k;         /* bf16 [Hkv][r][D]                                               */
+    const int32_t *seq_lens; /* [B]: the current token is at position N_b - 1                  */
+    const uint8_t *head_mask;/* [Hkv], HOST: heads to produce (NULL: every head)               */
+    void *q_idx;             /* fp16 [B][Hkv][r], written for the selected heads               */
+    void *k_idx;             /* fp16 [B][Hkv][max_ctx][r]: row N_b - 1 of the selected heads   */
+} rtp_indexer_io;
+
+RTP_API rtp_status rtp_indexer_append(rtp_handle *h, const rtp_indexer_io *io, void *stream);
+
 /* Dense full attention over all N_b tokens for every KV head (top_p, q_idx, k_idx and the mask
  * are ignored). The speedup denominator: same caches, same kernels, no selection. */
 RTP_API rtp_status rtp_dense_decode(rtp_handle *h, const rtp_layer_io *io, void *stream);

@@ -143,6 +143,53 @@ def test_selection_ranges_beyond_on_chip_capacity():
     _run(p, exact=False)
 
 
+@pytest.mark.parametrize("B,Hq,Hkv", [(1, 32, 4), (8, 32, 4), (3, 16, 8), (2, 8, 8)])
+def test_indexer_append_matches_oracle(B, Hq, Hkv):
+    """rtp_indexer_append: q_idx and the new k_idx row agree with the fp64 oracle rounded to
+    fp16 (fp32 accumulation may differ by one fp16 unit next to a rounding boundary); only row
+    N_b - 1 of the selected heads changes and q_idx of unselected heads is left alone."""
+    import oracle
+    G, D, r, max_ctx = Hq // Hkv, 128, 16, 300
+    g = torch.Generator(device=DEV).manual_seed(B * 100 + Hq + Hkv)
+    bf = lambda *sh, sd=1.0: (torch.randn(*sh, generator=g, device=DEV) * sd).to(torch.bfloat16)
+    q_pre, k_pre = bf(B, Hq, D), bf(B, Hkv, D)
+    w_q, w_k = bf(Hkv, r, G * D, sd=0.03), bf(Hkv, r, D, sd=0.1)
+    seq = torch.tensor([max_ctx - 7 * b for b in range(B)], dtype=torch.int32, device=DEV)
+    k_idx = torch.randn(B, Hkv, max_ctx, r, generator=g, device=DEV).to(torch.float16)
+    q_idx = torch.full((B, Hkv, r), 7.0, dtype=torch.float16, device=DEV)
+    k_before, q_before = k_idx.clone(), q_idx.clone()
+    mask = np.array([(h + 1) % 3 != 0 for h in range(Hkv)], np.uint8)
+    p = W.custom(batch=B, num_q_heads=Hq, num_kv_heads=Hkv, seq_lens=seq.tolist(),
+                 max_ctx=max_ctx, retrieval=[0] * Hkv, kinds=[[0] * Hkv] * B)
+    with make_handle(p) as h:
+        h.indexer_append(q_pre, k_pre, w_q, w_k, seq, q_idx, k_idx, head_mask=mask)
+        torch.cuda.synchronize()
+        assert h.device_status() == 0
+    qi, ki = oracle.indexer_project(W.to_host_u16(q_pre), W.to_host_u16(k_pre),
+                                    W.to_host_u16(w_q), W.to_host_u16(w_k))
+    ulp = lambda a, b: np.abs(a.astype(np.int32) - b.astype(np.int32))
+    gq = q_idx.cpu().numpy().view(np.uint16).astype(np.int16)
+    gk = k_idx.cpu().numpy().view(np.uint16)
+    exact = total = 0
+    for b in range(B):
+        n = int(seq[b])
+        for hh in range(Hkv):
+            if not mask[hh]:
+                assert torch.equal(q_idx[b, hh], q_before[b, hh])
+                assert torch.equal(k_idx[b, hh], k_before[b, hh])
+                continue
+            want_q = qi[b, hh].astype(np.float16).view(np.int16)
+            want_k = ki[b, hh].astype(np.float16).view(np.int16)
+            got_k = gk[b, hh, n - 1].astype(np.int16)
+            assert ulp(gq[b, hh], want_q).max() <= 1 and ulp(got_k, want_k).max() <= 1
+            exact += int((gq[b, hh] == want_q).sum() + (got_k == want_k).sum())
+            total += 2 * r
+            others = torch.ones(max_ctx, dtype=torch.bool)
+            others[n - 1] = False
+            assert torch.equal(k_idx[b, hh][others.to(DEV)], k_before[b, hh][others.to(DEV)])
+    assert exact >= 0.97 * total
+
+
 def test_dense_decode_matches_oracle():
     p = W.custom(batch=2, num_q_heads=32, num_kv_heads=4, seq_lens=[33000, 7],
                  max_ctx=33000, retrieval=[1, 0, 0, 0],
