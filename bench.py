@@ -113,18 +113,20 @@ def step_bytes(plan, sel_counts) -> tuple[int, int, int]:
     return idx + att, att, idx
 
 
-def cpu_sample_layers(plan):
-    """A bounded sample of the workload for the CPU oracle: one layer with a broad (diffuse or
-    flat) retrieval query, one with a concentrated one and one with local heads only."""
+def cpu_sample_layers(plan, per_kind: int = 2):
+    """A bounded sample of the workload for the CPU oracle (about 10 s of fp64 work at 1M
+    context): per_kind layers with a broad (diffuse or flat) retrieval query, with a
+    concentrated one and with local heads only."""
     from head_wise_sparse_retrieval_b200 import workloads as W
     pick = []
     for cond in (lambda l: ((plan.kind[l] == W.KIND_DIFFUSE) | (plan.kind[l] == W.KIND_FLAT)).any(),
                  lambda l: (plan.kind[l] == W.KIND_CONC).any(),
                  lambda l: not plan.retrieval[l].any()):
+        got = 0
         for l in range(plan.num_layers):
-            if cond(l) and l not in pick:
+            if got < per_kind and cond(l) and l not in pick:
                 pick.append(l)
-                break
+                got += 1
     return pick or [0]
 
 
