@@ -227,12 +227,15 @@ cudaError_t launch_one(rtp_handle* h, int kind, Kernel k, dim3 grid, dim3 block,
   return e;
 }
 
-rtp_status enqueue_layer(rtp_handle* h, const LayerArgs& a0, cudaStream_t s, int top_k = 0) {
+rtp_status enqueue_layer(rtp_handle* h, const LayerArgs& a0, cudaStream_t s, int top_k = 0,
+                         unsigned long long wait_ns = kWaitLimitNs, int withhold_cta = -1) {
   cudaError_t e;
   if (!a0.dense && a0.nret > 0) {
     SelectArgs x;
     x.top_k = top_k;
     x.hist_cnt = h->hist_cnt;
+    x.wait_ns = wait_ns;
+    x.withhold_cta = withhold_cta;
     // the ranges are at most ceil(B * nret * max_ctx / grid) tokens: on chip when that fits
     const long long worst = (long long)a0.B * a0.nret * a0.max_ctx;
     const bool fits = (worst + h->select_grid - 1) / h->select_grid <= kScoreCap;
@@ -240,6 +243,7 @@ rtp_status enqueue_layer(rtp_handle* h, const LayerArgs& a0, cudaStream_t s, int
                    dim3(kSelThreads), h->select_smem, s, true, a0, h->ws, x);
     if (e != cudaSuccess) return cuda_fail(e, "select_kernel launch");
   }
+  if (withhold_cta >= 0) return RTP_OK;  // self-test: the selection alone
   const LayerArgs& a = a0;
   e = launch_one(h, 1, attend_kernel, dim3(h->attend_grid), dim3(kAttendThreads), h->attend_smem,
                  s, false, a, h->ws);
@@ -485,6 +489,32 @@ rtp_status rtp_indexer_append(rtp_handle* h, const rtp_indexer_io* io, void* str
   cfg.numAttrs = 1;
   cudaError_t e = cudaLaunchKernelEx(&cfg, indexer_kernel, x);
   return e == cudaSuccess ? ok() : cuda_fail(e, "indexer_kernel launch");
+}
+
+rtp_status rtp_selftest_wait_timeout(rtp_handle* h, int layer, const rtp_layer_io* io,
+                                     uint64_t wait_ns, void* stream) {
+  if (!h) return fail(RTP_ERR_INVALID_ARG, "handle is NULL");
+  if (layer < 0 || layer >= h->cfg.num_layers)
+    return fail(RTP_ERR_INVALID_ARG, "layer %d outside [0, %d)", layer, h->cfg.num_layers);
+  if (!io || !io->retrieval_mask) return fail(RTP_ERR_INVALID_ARG, "io or its mask is NULL");
+  if (wait_ns < 1000 || wait_ns > 1000000000ull)
+    return fail(RTP_ERR_INVALID_ARG, "wait_ns must be in [1 us, 1 s]");
+  LayerArgs a = make_args(h, io);
+  a.nret = 0;
+  for (int kvh = 0; kvh < a.Hkv; ++kvh) {
+    if (io->retrieval_mask[kvh]) {
+      a.slot_of_kvh[kvh] = (short)a.nret;
+      a.ret_kvh[a.nret++] = (short)kvh;
+    }
+  }
+  if (a.nret == 0) return fail(RTP_ERR_INVALID_ARG, "the mask has no retrieval head");
+  rtp_status st = check_io(h, io, true);
+  if (st != RTP_OK) return st;
+  DeviceGuard guard(h->device);
+  st = enqueue_layer(h, a, static_cast<cudaStream_t>(stream), io->top_k, wait_ns, 0);
+  if (st != RTP_OK) return st;
+  h->last_valid = false;  // its selection lists are not meaningful
+  return ok();
 }
 
 rtp_status rtp_dense_decode(rtp_handle* h, const rtp_layer_io* io, void* stream) {

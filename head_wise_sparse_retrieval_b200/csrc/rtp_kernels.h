@@ -35,6 +35,8 @@ struct Workspace {
 struct SelectArgs {
   int top_k;                      // > 0: b* by token count (fixed top-k) instead of mass
   unsigned* hist_cnt;             // [kHistCopies][slots][256] tokens per bin (top-k only)
+  unsigned long long wait_ns;     // limit of every grid-barrier wait
+  int withhold_cta;               // self-test: CTA that skips its first arrival, else -1
 };
 
 struct LayerArgs {

@@ -115,17 +115,21 @@ __device__ __forceinline__ T block_suffix_sum(T v, T* red) {
 // flips once per barrier: CTA 0 adds 2^31 - (P - 1), every other CTA adds 1, so the low 31
 // bits (0 between barriers) reach 2^31 and carry into the top bit exactly at the last arrival.
 // The add has release semantics (it publishes the CTA's writes) and the polling load acquire
-// semantics. The wait gives up after kWaitLimitNs, sets kDevWaitTimeout and makes later
+// semantics. The wait gives up after limit_ns, sets kDevWaitTimeout and makes later
 // barriers of the CTA return at once, so the kernel ends (the host then clears the counter).
-__device__ void grid_barrier(unsigned* bar, unsigned* status, int* aborted) {
+// withhold: a CTA index that does not arrive (self-test of the bounded wait), or -1.
+__device__ void grid_barrier(unsigned* bar, unsigned* status, int* aborted,
+                             unsigned long long limit_ns, int withhold) {
   __syncthreads();
-  if (threadIdx.x == 0 && !*aborted) {
+  if (threadIdx.x == 0 && !*aborted && (int)blockIdx.x == withhold) {
+    *aborted = 1;  // never arrives: every other CTA's wait runs out
+  } else if (threadIdx.x == 0 && !*aborted) {
     const unsigned inc = (blockIdx.x == 0) ? 0x80000000u - (gridDim.x - 1u) : 1u;
     const unsigned old = atomic_add_acq_rel_gpu(bar, inc);
     const unsigned long long t0 = global_ns();
     unsigned it = 0;
     while (((ld_acquire_gpu(bar) ^ old) & 0x80000000u) == 0u) {
-      if ((++it & 255u) == 0 && global_ns() - t0 > kWaitLimitNs) {
+      if ((++it & 255u) == 0 && global_ns() - t0 > limit_ns) {
         atomicOr(status, kDevWaitTimeout);
         *aborted = 1;
         break;
@@ -308,7 +312,7 @@ __device__ __forceinline__ void select_body(const LayerArgs& a, const Workspace&
       if (tid == 0) w.cta_max[(size_t)s * gridDim.x + blockIdx.x] = mx;
     }
   }
-  grid_barrier(w.grid_bar, w.status, &aborted);
+  grid_barrier(w.grid_bar, w.status, &aborted, x.wait_ns, x.withhold_cta);
 
   // ---- phase 2: mass histogram and token counts of this CTA's segments ---------------------
   if (active) {
@@ -367,7 +371,7 @@ __device__ __forceinline__ void select_body(const LayerArgs& a, const Workspace&
       __syncthreads();
     }
   }
-  grid_barrier(w.grid_bar, w.status, &aborted);
+  grid_barrier(w.grid_bar, w.status, &aborted, x.wait_ns, -1);
 
   // ---- phase 3: b*, offsets and the dense selected list -----------------------------------
   if (active) {
@@ -440,7 +444,13 @@ __device__ __forceinline__ void select_body(const LayerArgs& a, const Workspace&
         const unsigned lt = (1u << lane) - 1u;
 #pragma unroll
         for (int k = 0; k < kPerThread; ++k) {
-          if (bal[k] & (1u << lane)) out[at + __popc(bal[k] & lt)] = wb + 32 * k + lane;
+          // in range by construction; after an abandoned barrier the offsets may be stale, so
+          // the row's capacity is still checked
+          const int dst = at + __popc(bal[k] & lt);
+          if (bal[k] & (1u << lane)) {
+            if ((unsigned)dst < (unsigned)w.ld) out[dst] = wb + 32 * k + lane;
+            else atomicOr(w.status, kDevBadIndex);
+          }
           at += __popc(bal[k]);
         }
         base += all;

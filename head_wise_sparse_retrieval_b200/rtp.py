@@ -25,7 +25,7 @@ EXPORTS = ("rtp_config_default", "rtp_workspace_bytes", "rtp_create", "rtp_destr
            "rtp_decode_step", "rtp_dense_decode", "rtp_decode_step_host", "rtp_get_selection",
            "rtp_get_threshold", "rtp_get_device_status", "rtp_status_string", "rtp_last_error",
            "rtp_profile_enable", "rtp_profile_read", "rtp_window_attention_noalloc",
-           "rtp_indexer_append")
+           "rtp_indexer_append", "rtp_selftest_wait_timeout")
 NOALLOC_MAX_HEADS = 64
 KERNEL_CLASSES = ("select", "attend", "merge", "reserved3")
 
@@ -109,6 +109,8 @@ def load(path: str = LIB_PATH):
     L.rtp_window_attention_noalloc.restype = ctypes.c_int
     L.rtp_indexer_append.argtypes = [vp, ctypes.POINTER(IndexerIO), vp]
     L.rtp_indexer_append.restype = ctypes.c_int
+    L.rtp_selftest_wait_timeout.argtypes = [vp, i, ctypes.POINTER(LayerIO), ctypes.c_uint64, vp]
+    L.rtp_selftest_wait_timeout.restype = ctypes.c_int
     L.rtp_status_string.argtypes = [i]
     L.rtp_status_string.restype = ctypes.c_char_p
     L.rtp_last_error.argtypes = []
@@ -241,6 +243,14 @@ class Handle:
                        _ptr(q_idx), _ptr(k_idx))
         _check(load().rtp_indexer_append(self._h, ctypes.byref(io), _stream_ptr(stream)),
                "rtp_indexer_append")
+
+    def selftest_wait_timeout(self, layer_idx: int, layer: Layer, mask, top_p: float, out,
+                              wait_ns: int, stream=None):
+        """rtp_selftest_wait_timeout: the layer's selection with one barrier arrival withheld."""
+        io = self._io(layer, mask, top_p, out)
+        _check(load().rtp_selftest_wait_timeout(self._h, layer_idx, ctypes.byref(io),
+                                                int(wait_ns), _stream_ptr(stream)),
+               "rtp_selftest_wait_timeout")
 
     def selection(self, b: int, kvh: int) -> np.ndarray:
         """Ascending positions selected for (b, kvh) by the last decode_step."""

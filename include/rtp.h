@@ -210,6 +210,17 @@ RTP_API rtp_status rtp_profile_enable(rtp_handle *h, int enable);
  * into ms[4] and launches[4] (overwritten), and empties the pool. */
 RTP_API rtp_status rtp_profile_read(rtp_handle *h, double *ms, int64_t *launches);
 
+/* Self-test of failure detection without a GPU fault: enqueues the selection of one layer (as
+ * rtp_decode_step would, attention not launched) with CTA 0 withholding its arrival at the
+ * first grid barrier and every barrier wait limited to wait_ns (1 us .. 1 s). The other CTAs'
+ * waits run out, the launch ends on its own, and RTP_DEV_WAIT_TIMEOUT is set in the device
+ * status word; rtp_get_device_status reports it and clears the barrier state, after which the
+ * handle decodes normally. The selection lists it leaves are not meaningful (the debug
+ * getters refuse them). The pages describe no such call. Errors: RTP_ERR_INVALID_ARG for a
+ * mask without retrieval heads or wait_ns out of range, otherwise as rtp_decode_step. */
+RTP_API rtp_status rtp_selftest_wait_timeout(rtp_handle *h, int layer, const rtp_layer_io *io,
+                                             uint64_t wait_ns, void *stream);
+
 /* Reads and clears the device status word (RTP_DEV_* bits) after synchronising the device.
  * After RTP_DEV_WAIT_TIMEOUT it also resets the selection kernel's grid-barrier counter, so
  * that later calls on the handle start from a clean barrier. Returns RTP_ERR_DEVICE_STATUS

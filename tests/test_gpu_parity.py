@@ -312,6 +312,25 @@ def test_inputs_ready_chaining_matches_strict_ordering():
         assert torch.equal(res[True][1][l], res[False][1][l])
 
 
+def test_bounded_wait_runs_out_and_is_reported():
+    """Failure detection without a GPU fault: one selection CTA withholds its barrier arrival,
+    the other CTAs' bounded waits (2 ms here) run out, the launch ends by itself and the status
+    word reports the timeout; the handle then decodes normally."""
+    p = W.plan("one_layer", query="conc")
+    li = W.make_layer(p, 0, DEV)
+    with make_handle(p) as h:
+        out = torch.empty((1, 32, 128), dtype=torch.float32, device=DEV)
+        assert h.device_status() == 0
+        h.selftest_wait_timeout(0, rtp.layer_from(li), p.retrieval[0], p.top_p, out,
+                                wait_ns=2_000_000)
+        code = h.device_status()
+        assert code & rtp.DEV_WAIT_TIMEOUT, hex(code)
+        assert h.device_status() == 0  # read and cleared
+        with pytest.raises(rtp.RtpError):
+            h.selection(0, 0)  # the self-test's lists are not meaningful
+        check_layer(h, p, li, 0)
+
+
 def test_bad_seq_len_is_reported_not_faulted():
     p = W.custom(batch=2, num_q_heads=8, num_kv_heads=1, seq_lens=[100, 50], max_ctx=128,
                  retrieval=[1], kinds=[[W.KIND_CONC]] * 2, n_needles=[[2]] * 2, seed=14)
