@@ -1,8 +1,8 @@
 // rtp_device.cuh -- device-side building blocks shared by the kernels of librtp (sm_100a).
 //
-// Inline PTX wrappers for: programmatic dependent launch, mbarriers with bounded waits,
-// asynchronous copies global -> shared (cp.async, 1-D bulk), ldmatrix, movmatrix and the
-// warp-level bf16 MMA used to spare the FP32 pipes in the gather kernel.
+// Inline PTX wrappers for: programmatic dependent launch, GPU-scope atomics and acquire loads,
+// asynchronous copies global -> shared (cp.async), ldmatrix, movmatrix and the warp-level
+// bf16 MMA used to spare the FP32 pipes in the gather kernel.
 #pragma once
 
 #include <cstdint>
@@ -20,7 +20,6 @@ constexpr int kMaxGroup = 8;             // query heads per KV head handled by o
 // a partial of one KV head's attention: o[8][128] (unnormalised), then m[8] (log2 domain), l[8]
 constexpr int kPartO = kMaxGroup * kHeadDim;
 constexpr int kPartFloats = kPartO + 2 * kMaxGroup;
-constexpr double kFixedOne = 1099511627776.0;  // 2^40: fixed-point unit of histogram masses
 
 // Device status bits (mirrors include/rtp.h).
 constexpr unsigned kDevBadSeqlen = 0x1u;
@@ -73,77 +72,10 @@ __device__ __forceinline__ unsigned long long global_ns() {
   return t;
 }
 
-// ---- shared-memory addresses and mbarriers ------------------------------------------------
+// ---- shared memory and asynchronous copies -----------------------------------------------
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
-}
-
-__device__ __forceinline__ void mbar_init(uint64_t* bar, unsigned count) {
-  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count)
-               : "memory");
-}
-
-__device__ __forceinline__ void fence_mbar_init() {
-  asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
-}
-
-__device__ __forceinline__ void fence_proxy_async_smem() {
-  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-}
-
-__device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
-  asm volatile("{\n\t.reg .b64 st;\n\tmbarrier.arrive.shared::cta.b64 st, [%0];\n\t}" ::"r"(
-                   smem_u32(bar))
-               : "memory");
-}
-
-__device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* bar, unsigned bytes) {
-  asm volatile(
-      "{\n\t.reg .b64 st;\n\tmbarrier.arrive.expect_tx.shared::cta.b64 st, [%0], %1;\n\t}" ::"r"(
-          smem_u32(bar)),
-      "r"(bytes)
-      : "memory");
-}
-
-__device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, unsigned parity) {
-  uint32_t ok;
-  asm volatile(
-      "{\n\t.reg .pred p;\n\tmbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
-      "selp.u32 %0, 1, 0, p;\n\t}"
-      : "=r"(ok)
-      : "r"(smem_u32(bar)), "r"(parity)
-      : "memory");
-  return ok != 0;
-}
-
-// Waits for the phase of `parity` to complete. Gives up after kWaitLimitNs, sets
-// kDevWaitTimeout in *status and raises *abort_flag (shared) so that later waits of the CTA
-// return at once: control flow stays identical across warps and the kernel ends.
-__device__ __forceinline__ void mbar_wait_bounded(uint64_t* bar, unsigned parity,
-                                                  unsigned* status, volatile int* abort_flag) {
-  if (mbar_try_wait(bar, parity)) return;
-  const unsigned long long t0 = global_ns();
-  for (unsigned it = 0;; ++it) {
-    if (*abort_flag) return;
-    if (mbar_try_wait(bar, parity)) return;
-    if ((it & 255u) == 255u && global_ns() - t0 > kWaitLimitNs) {
-      atomicOr(status, kDevWaitTimeout);
-      *abort_flag = 1;
-      return;
-    }
-  }
-}
-
-// 1-D bulk copy global -> shared of `bytes` (multiple of 16, both addresses 16-byte aligned),
-// completing `bytes` of transaction count on `bar`. L2 policy: evict-first (read-once data).
-__device__ __forceinline__ void bulk_g2s(void* smem_dst, const void* gmem_src, unsigned bytes,
-                                         uint64_t* bar, uint64_t policy) {
-  asm volatile(
-      "cp.async.bulk.shared::cta.global.mbarrier::complete_tx::bytes.L2::cache_hint"
-      " [%0], [%1], %2, [%3], %4;" ::"r"(smem_u32(smem_dst)),
-      "l"(gmem_src), "r"(bytes), "r"(smem_u32(bar)), "l"(policy)
-      : "memory");
 }
 
 __device__ __forceinline__ uint64_t l2_policy_evict_first() {
@@ -166,10 +98,6 @@ __device__ __forceinline__ void cp_async_commit() {
 template <int N>
 __device__ __forceinline__ void cp_async_wait() {
   asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
-}
-
-__device__ __forceinline__ void named_barrier_sync(int id, int nthreads) {
-  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
 }
 
 // ---- warp-level matrix fragments ----------------------------------------------------------
