@@ -348,7 +348,6 @@ def main():
         raise SystemExit(f"device status 0x{status:x} after the eager step")
     sel = [c.cpu().numpy() for c in cnts]
     total_bytes, attend_bytes, idx_bytes = step_bytes(plan, sel)
-    launches_per_step = sum(3 if plan.retrieval[l].any() else 2 for l in range(L))  # [select,] attend, merge
 
     # capture the whole step as one CUDA graph
     g = torch.cuda.CUDAGraph()
@@ -393,6 +392,9 @@ def main():
     h.profile(False)
     kern = {k: {"ms_total_per_step": v[0] / prof_steps, "launches_per_step": v[1] / prof_steps}
             for k, v in acc.items() if v[1]}
+    # launches of the step as counted by the library's per-launch events ([select,] attend
+    # [, merge] per layer: the merge folds into the attention launch when its grid fits at once)
+    launches_per_step = round(sum(v[1] for v in acc.values()) / prof_steps)
     att_ms = acc["attend"][0] / max(acc["attend"][1], 1)
     att_bytes_per_launch = attend_bytes / L
     hbm, peak_kind = _peaks()
