@@ -278,6 +278,8 @@ def main():
     ap.add_argument("--single-layer", type=int, default=None,
                     help="profiling case: only this layer of the workload, decoded --reps times")
     ap.add_argument("--reps", type=int, default=3)
+    ap.add_argument("--single-launch", action="store_true",
+                    help="--single-layer: run the layer as one fused launch")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
 
@@ -308,7 +310,8 @@ def main():
         out = torch.empty((plan.batch, plan.num_q_heads, 128), dtype=torch.float32, device=dev)
         cnt = torch.empty((plan.batch, plan.num_kv_heads), dtype=torch.int32, device=dev)
         for _ in range(args.reps):
-            h.decode_step(l, rtp.layer_from(li), plan.retrieval[l], plan.top_p, out, cnt)
+            h.decode_step(l, rtp.layer_from(li), plan.retrieval[l], plan.top_p, out, cnt,
+                          single_launch=args.single_launch)
         torch.cuda.synchronize()
         status = h.device_status()
         h.close()
@@ -407,11 +410,11 @@ def main():
 
     # the same step at other p (the 1M-context configuration sweeps p over 0.8 / 0.9 / 0.95)
     # and with the fixed top-k of the pages' top-k / top-p comparison (2k / 4k / 16k)
-    def time_variant(pv, kv, ready=False):
+    def time_variant(pv, kv, ready=False, single=False):
         def run():
             for l in range(L):
                 h.decode_step(l, views[l], plan.retrieval[l], pv, outs[l], cnts[l],
-                              stream=stream, top_k=kv, inputs_ready=ready)
+                              stream=stream, top_k=kv, inputs_ready=ready, single_launch=single)
         with torch.cuda.stream(stream):
             run()
         torch.cuda.synchronize()
@@ -451,6 +454,11 @@ def main():
     # the same step with rtp_layer_io.inputs_ready: every input is resident before the step,
     # so each layer's scoring / local attention streams while the previous launch drains
     chained = time_variant(plan.top_p, 0, ready=True)
+    # the same step with every layer as one fused launch (rtp_layer_io.single_launch)
+    try:
+        single = time_variant(plan.top_p, 0, single=True)
+    except rtp.RtpError as e:  # shapes beyond the single-launch limits
+        single = {"unsupported": str(e)}
 
     # indexer production of one layer (q_idx and the new k_idx row of every KV head), timed as a
     # CUDA graph of 100 calls; W is random (no trained weights), the row goes to a scratch cache
@@ -584,6 +592,7 @@ def main():
         "p_sweep": p_sweep,
         "k_sweep": k_sweep,
         "chained": chained,
+        "single_launch": single,
         "indexer_append": indexer,
         "dense": dense,
         "e2e": e2e,

@@ -24,6 +24,11 @@ struct rtp_handle {
   size_t ws_bytes = 0;
   Workspace ws{};
   unsigned* hist_cnt = nullptr;  // selection token counts per bin (fixed top-k)
+  // single-launch layers (fused_layer_kernel): one CTA per SM, when B * Hkv <= kFusedMaxHeads
+  bool fused_ok = false;
+  int fused_grid = 0;
+  size_t fused_smem = 0;
+  FusedArgs fx{};
   // staging for rtp_decode_step_host
   void* stage_q = nullptr;
   void* stage_qidx = nullptr;
@@ -33,6 +38,7 @@ struct rtp_handle {
   bool last_valid = false;
   cudaStream_t last_stream = nullptr;
   int last_nret = 0;
+  bool last_fused = false;  // the selection is in the masks, not the position lists
   short last_slot_of_kvh[kMaxKvHeads];
   // rtp_decode_step_host replays the layer sequence as a CUDA graph, captured once per
   // (layer count, p, cache pointers, masks) on a stream of the handle
@@ -111,9 +117,10 @@ struct WsPlan {
 };
 
 // Byte offsets of the workspace arrays (each 256-byte aligned).
-WsPlan plan_workspace(const rtp_config* c, int attend_grid, int select_grid) {
+WsPlan plan_workspace(const rtp_config* c, int attend_grid, int select_grid, int fused_grid) {
   const size_t slots = (size_t)c->batch * c->num_kv_heads;
   const size_t nmax = round_up((size_t)c->max_ctx, 64);  // per-slot stride (16-byte loads)
+  const bool fused = slots <= (size_t)kFusedMaxHeads;
   const size_t sizes[] = {
       slots * nmax * 4,                      // 0 scores
       slots * (size_t)select_grid * 4,       // 1 cta_max
@@ -132,6 +139,9 @@ WsPlan plan_workspace(const rtp_config* c, int attend_grid, int select_grid) {
       ((size_t)attend_grid + slots) * kPartFloats * 4,  // 14 partials
       256,                                   // 15 status
       (size_t)kHistCopies * slots * kBins * 4,  // 16 hist_cnt
+      fused ? slots * 4 : 0,                 // 17 smax_key
+      fused ? slots * (nmax / 64) * 8 : 0,   // 18 sel_bits
+      fused ? (slots * fused_grid + fused_grid + slots) * kPartFloats * 4 : 0,  // 19 pieces
   };
   WsPlan p{};
   size_t at = 0;
@@ -227,6 +237,27 @@ cudaError_t launch_one(rtp_handle* h, int kind, Kernel k, dim3 grid, dim3 block,
   return e;
 }
 
+// Whether the layer fits the single-launch kernel: B * Hkv within its tables, and the ownership
+// tiles of the worst case (every N_b = max_ctx) within each CTA's on-chip share.
+bool fused_fits(const rtp_handle* h, const LayerArgs& a) {
+  if (!h->fused_ok || a.dense) return false;
+  const long long tiles =
+      (long long)a.B * a.nret * ((a.max_ctx + kFusedOwnTok - 1) / kFusedOwnTok);
+  return (tiles + h->fused_grid - 1) / h->fused_grid <= kFusedCapTiles;
+}
+
+rtp_status enqueue_fused(rtp_handle* h, const LayerArgs& a, cudaStream_t s, int top_k) {
+  if (!fused_fits(h, a))
+    return fail(RTP_ERR_UNSUPPORTED,
+                "single launch: needs B*Hkv <= %d and B*nret*ceil(max_ctx/64) <= %d*%d",
+                kFusedMaxHeads, h->fused_grid, kFusedCapTiles);
+  FusedArgs f = h->fx;
+  f.top_k = top_k;
+  const cudaError_t e = launch_one(h, 3, fused_layer_kernel, dim3(h->fused_grid),
+                                   dim3(kFusedThreads), h->fused_smem, s, true, a, h->ws, f);
+  return e == cudaSuccess ? RTP_OK : cuda_fail(e, "fused_layer_kernel launch");
+}
+
 rtp_status enqueue_layer(rtp_handle* h, const LayerArgs& a0, cudaStream_t s, int top_k = 0,
                          unsigned long long wait_ns = kWaitLimitNs, int withhold_cta = -1) {
   cudaError_t e;
@@ -297,7 +328,7 @@ size_t rtp_workspace_bytes(const rtp_config* cfg) {
   int dev = 0, sms = 148;
   if (cudaGetDevice(&dev) == cudaSuccess)
     cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-  return plan_workspace(cfg, sms * kAttendCtasPerSm, sms * kMaxSelectCtasPerSm).total;
+  return plan_workspace(cfg, sms * kAttendCtasPerSm, sms * kMaxSelectCtasPerSm, sms).total;
 }
 
 rtp_status rtp_create(const rtp_config* cfg, int device, rtp_handle** out) {
@@ -341,7 +372,8 @@ rtp_status rtp_create(const rtp_config* cfg, int device, rtp_handle** out) {
   }
   if (sel_per_sm > kMaxSelectCtasPerSm) sel_per_sm = kMaxSelectCtasPerSm;
   h->select_grid = h->num_sms * sel_per_sm;  // cooperative: every CTA resident at once
-  const WsPlan p = plan_workspace(cfg, h->attend_grid, h->select_grid);
+  h->fused_grid = h->num_sms;  // one CTA per SM
+  const WsPlan p = plan_workspace(cfg, h->attend_grid, h->select_grid, h->fused_grid);
   const size_t L = (size_t)cfg->num_layers, B = (size_t)cfg->batch;
   const size_t q_bytes = L * B * cfg->num_q_heads * kHeadDim * 2;
   const size_t qi_bytes = L * B * cfg->num_kv_heads * kIdxDim * 2;
@@ -383,6 +415,13 @@ rtp_status rtp_create(const rtp_config* cfg, int device, rtp_handle** out) {
   w.partials = reinterpret_cast<float*>(base + p.off[14]);
   w.status = reinterpret_cast<unsigned*>(base + p.off[15]);
   h->hist_cnt = reinterpret_cast<unsigned*>(base + p.off[16]);
+  h->fx.hist_cnt = h->hist_cnt;
+  h->fx.smax_key = reinterpret_cast<unsigned*>(base + p.off[17]);
+  h->fx.sel_bits = reinterpret_cast<unsigned long long*>(base + p.off[18]);
+  h->fx.partials = reinterpret_cast<float*>(base + p.off[19]);
+  h->fx.bar = w.grid_bar + kFusedBarWord;
+  h->fx.wait_ns = kWaitLimitNs;
+  h->fx.ldw = (int)(round_up((size_t)cfg->max_ctx, 64) / 64);
   w.ld = (int)round_up((size_t)cfg->max_ctx, 64);
   h->stage_q = base + stage_q_off;
   h->stage_qidx = base + stage_qi_off;
@@ -405,6 +444,22 @@ rtp_status rtp_create(const rtp_config* cfg, int device, rtp_handle** out) {
     cudaFree(h->ws_mem);
     delete h;
     return cuda_fail(e, "cudaFuncSetAttribute(attend_kernel)");
+  }
+  if ((long long)cfg->batch * cfg->num_kv_heads <= kFusedMaxHeads &&
+      fused_smem_bytes() <= (size_t)max_optin) {
+    h->fused_smem = fused_smem_bytes();
+    int per_sm = 0;
+    e = cudaFuncSetAttribute(fused_layer_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)h->fused_smem);
+    if (e == cudaSuccess)
+      e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, fused_layer_kernel,
+                                                        kFusedThreads, h->fused_smem);
+    if (e != cudaSuccess) {
+      cudaFree(h->ws_mem);
+      delete h;
+      return cuda_fail(e, "cudaFuncSetAttribute(fused_layer_kernel)");
+    }
+    h->fused_ok = per_sm >= 1;  // the grid is one CTA per SM, all resident at once
   }
   *out = h;
   return ok();
@@ -442,8 +497,10 @@ rtp_status rtp_decode_step(rtp_handle* h, int layer, const rtp_layer_io* io, voi
   if (st != RTP_OK) return st;
   DeviceGuard guard(h->device);
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  st = enqueue_layer(h, a, s, io->top_k);
+  const bool single = io->single_launch != 0;
+  st = single ? enqueue_fused(h, a, s, io->top_k) : enqueue_layer(h, a, s, io->top_k);
   if (st != RTP_OK) return st;
+  h->last_fused = single;
   h->last_valid = true;
   h->last_stream = s;
   h->last_nret = a.nret;
@@ -662,10 +719,21 @@ rtp_status rtp_get_selection(rtp_handle* h, int b, int kvh, int32_t* idx_out, in
   *count = total;
   if (cap <= 0) return ok();
   const int64_t k = total < cap ? total : cap;
+  if (h->last_fused) {  // expand the slot's tile masks (bit i of word t: token 64 t + i)
+    const int words = (n + kFusedOwnTok - 1) / kFusedOwnTok;
+    std::vector<unsigned long long> m((size_t)words);
+    e = cudaMemcpy(m.data(), h->fx.sel_bits + (size_t)slot * h->fx.ldw, (size_t)words * 8,
+                   cudaMemcpyDeviceToHost);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaMemcpy");
+    int64_t at = 0;
+    for (int t = 0; t < words && at < k; ++t)
+      for (int i = 0; i < 64 && at < k; ++i)
+        if ((m[(size_t)t] >> i) & 1ull) idx_out[at++] = t * kFusedOwnTok + i;
+    return ok();
+  }
   e = cudaMemcpy(idx_out, h->ws.sel_idx + (size_t)slot * h->ws.ld, (size_t)k * 4,
                  cudaMemcpyDeviceToHost);
   if (e != cudaSuccess) return cuda_fail(e, "cudaMemcpy");
-  (void)n;
   return ok();
 }
 
@@ -689,7 +757,11 @@ rtp_status rtp_get_device_status(rtp_handle* h, uint32_t* code) {
   if (e == cudaSuccess) e = cudaMemcpy(code, h->ws.status, 4, cudaMemcpyDeviceToHost);
   if (e == cudaSuccess) e = cudaMemset(h->ws.status, 0, 4);
   // a barrier that timed out leaves its counter mid-count: start the next launch from zero
-  if (e == cudaSuccess && (*code & kDevWaitTimeout)) e = cudaMemset(h->ws.grid_bar, 0, 4);
+  if (e == cudaSuccess && (*code & kDevWaitTimeout)) {
+    e = cudaMemset(h->ws.grid_bar, 0, (kFusedBarWord + 1) * 4);
+    if (e == cudaSuccess && h->fused_ok)  // a stopped single launch may leave maxima behind
+      e = cudaMemset(h->fx.smax_key, 0, (size_t)h->cfg.batch * h->cfg.num_kv_heads * 4);
+  }
   if (e != cudaSuccess) return cuda_fail(e, "reading the device status");
   if (*code) return fail(RTP_ERR_DEVICE_STATUS, "device status 0x%x", *code);
   return ok();

@@ -72,6 +72,34 @@ __device__ __forceinline__ unsigned long long global_ns() {
   return t;
 }
 
+// Grid-wide barrier of a cooperative launch (every CTA is resident), one counter whose top bit
+// flips once per barrier: CTA 0 adds 2^31 - (P - 1), every other CTA adds 1, so the low 31
+// bits (0 between barriers) reach 2^31 and carry into the top bit exactly at the last arrival.
+// The add has release semantics (it publishes the CTA's writes) and the polling load acquire
+// semantics. The wait gives up after limit_ns, sets kDevWaitTimeout and makes later
+// barriers of the CTA return at once, so the kernel ends (the host then clears the counter).
+// withhold: a CTA index that does not arrive (self-test of the bounded wait), or -1.
+__device__ inline void grid_barrier(unsigned* bar, unsigned* status, int* aborted,
+                                    unsigned long long limit_ns, int withhold) {
+  __syncthreads();
+  if (threadIdx.x == 0 && !*aborted && (int)blockIdx.x == withhold) {
+    *aborted = 1;  // never arrives: every other CTA's wait runs out
+  } else if (threadIdx.x == 0 && !*aborted) {
+    const unsigned inc = (blockIdx.x == 0) ? 0x80000000u - (gridDim.x - 1u) : 1u;
+    const unsigned old = atomic_add_acq_rel_gpu(bar, inc);
+    const unsigned long long t0 = global_ns();
+    unsigned it = 0;
+    while (((ld_acquire_gpu(bar) ^ old) & 0x80000000u) == 0u) {
+      if ((++it & 255u) == 0 && global_ns() - t0 > limit_ns) {
+        atomicOr(status, kDevWaitTimeout);
+        *aborted = 1;
+        break;
+      }
+    }
+  }
+  __syncthreads();
+}
+
 // ---- shared memory and asynchronous copies -----------------------------------------------
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {

@@ -57,6 +57,28 @@ struct LayerArgs {
                                   // preceding launch ends: kernels may read them before waiting
 };
 
+// Single-launch layer (fused_kernel.cu): selection, gather and merge in one cooperative launch
+// of one CTA per SM. The retrieval slots' tokens are owned in 64-token tiles dealt round-robin
+// to the CTAs; a CTA holds at most kFusedCapTiles of them on chip.
+constexpr int kFusedWarps = 8;
+constexpr int kFusedThreads = kFusedWarps * 32;
+constexpr int kFusedOwnTok = 64;                         // tokens per ownership tile
+constexpr int kFusedMaxHeads = 64;                       // B * Hkv of a single-launch layer
+constexpr int kFusedCapTiles = 448;                      // ownership tiles a CTA keeps on chip
+constexpr int kFusedBarWord = 64;                        // its grid_bar word (own cache line)
+struct FusedArgs {
+  int top_k;                      // > 0: b* by token count (fixed top-k)
+  unsigned* hist_cnt;             // [kHistCopies][slots][256] tokens per bin
+  unsigned* smax_key;             // [slots] order-preserving key of s_max; 0 between launches
+  unsigned long long* sel_bits;   // [slots][ldw] selection mask of each 64-token tile
+  float* partials;                // [slots * P + P + B*Hkv][kPartFloats] pieces
+  unsigned* bar;                  // grid-barrier counter of this kernel
+  unsigned long long wait_ns;     // limit of every grid-barrier wait
+  int ldw;                        // per-slot stride of sel_bits (words)
+};
+__global__ void fused_layer_kernel(const LayerArgs a, const Workspace w, const FusedArgs f);
+size_t fused_smem_bytes();
+
 // Indexer production at decode (indexer_kernel.cu).
 struct IndexerArgs {
   const __nv_bfloat16* q_pre;     // [B][Hq][128]

@@ -111,34 +111,6 @@ __device__ __forceinline__ T block_suffix_sum(T v, T* red) {
   return x + after;
 }
 
-// Grid-wide barrier of a cooperative launch (every CTA is resident), one counter whose top bit
-// flips once per barrier: CTA 0 adds 2^31 - (P - 1), every other CTA adds 1, so the low 31
-// bits (0 between barriers) reach 2^31 and carry into the top bit exactly at the last arrival.
-// The add has release semantics (it publishes the CTA's writes) and the polling load acquire
-// semantics. The wait gives up after limit_ns, sets kDevWaitTimeout and makes later
-// barriers of the CTA return at once, so the kernel ends (the host then clears the counter).
-// withhold: a CTA index that does not arrive (self-test of the bounded wait), or -1.
-__device__ void grid_barrier(unsigned* bar, unsigned* status, int* aborted,
-                             unsigned long long limit_ns, int withhold) {
-  __syncthreads();
-  if (threadIdx.x == 0 && !*aborted && (int)blockIdx.x == withhold) {
-    *aborted = 1;  // never arrives: every other CTA's wait runs out
-  } else if (threadIdx.x == 0 && !*aborted) {
-    const unsigned inc = (blockIdx.x == 0) ? 0x80000000u - (gridDim.x - 1u) : 1u;
-    const unsigned old = atomic_add_acq_rel_gpu(bar, inc);
-    const unsigned long long t0 = global_ns();
-    unsigned it = 0;
-    while (((ld_acquire_gpu(bar) ^ old) & 0x80000000u) == 0u) {
-      if ((++it & 255u) == 0 && global_ns() - t0 > limit_ns) {
-        atomicOr(status, kDevWaitTimeout);
-        *aborted = 1;
-        break;
-      }
-    }
-  }
-  __syncthreads();
-}
-
 // Slot sizes (clamped sequence lengths) and their prefix sums into soff[0 .. S]. report: flag
 // out-of-range lengths in the status word.
 __device__ void slot_offsets(const LayerArgs& a, int S, long long* soff, unsigned* status,

@@ -27,7 +27,7 @@ EXPORTS = ("rtp_config_default", "rtp_workspace_bytes", "rtp_create", "rtp_destr
            "rtp_profile_enable", "rtp_profile_read", "rtp_window_attention_noalloc",
            "rtp_indexer_append", "rtp_selftest_wait_timeout")
 NOALLOC_MAX_HEADS = 64
-KERNEL_CLASSES = ("select", "attend", "merge", "reserved3")
+KERNEL_CLASSES = ("select", "attend", "merge", "fused")
 
 
 class RtpError(RuntimeError):
@@ -69,7 +69,7 @@ class LayerIO(ctypes.Structure):
         ("v_cache", ctypes.c_void_p), ("k_idx", ctypes.c_void_p), ("seq_lens", ctypes.c_void_p),
         ("retrieval_mask", ctypes.POINTER(ctypes.c_uint8)), ("top_p", ctypes.c_float),
         ("out", ctypes.c_void_p), ("sel_count", ctypes.c_void_p), ("top_k", ctypes.c_int32),
-        ("inputs_ready", ctypes.c_int32),
+        ("inputs_ready", ctypes.c_int32), ("single_launch", ctypes.c_int32),
     ]
 
 
@@ -192,22 +192,24 @@ class Handle:
             pass
 
     def _io(self, layer: Layer, mask, top_p: float, out, sel_count=None, top_k: int = 0,
-            inputs_ready: bool = False) -> LayerIO:
+            inputs_ready: bool = False, single_launch: bool = False) -> LayerIO:
         m = np.ascontiguousarray(np.asarray(mask, dtype=np.uint8))
         assert m.shape == (self.cfg.num_kv_heads,)
         io = LayerIO(_ptr(layer.q), _ptr(layer.q_idx), _ptr(layer.k_cache), _ptr(layer.v_cache),
                      _ptr(layer.k_idx), _ptr(layer.seq_lens),
                      m.ctypes.data_as(ctypes.POINTER(ctypes.c_uint8)), float(top_p), _ptr(out),
-                     _ptr(sel_count), int(top_k), 1 if inputs_ready else 0)
+                     _ptr(sel_count), int(top_k), 1 if inputs_ready else 0,
+                     1 if single_launch else 0)
         io._mask = m  # keep the host mask alive for the duration of the call
         return io
 
     def decode_step(self, layer_idx: int, layer: Layer, mask, top_p: float, out,
-                    sel_count=None, stream=None, top_k: int = 0, inputs_ready: bool = False):
+                    sel_count=None, stream=None, top_k: int = 0, inputs_ready: bool = False,
+                    single_launch: bool = False):
         """rtp_decode_step: enqueue one layer on `stream` (default: torch's current stream).
         top_k > 0 selects by fixed top-k through the histogram instead of top-p;
-        inputs_ready: see rtp_layer_io.inputs_ready."""
-        io = self._io(layer, mask, top_p, out, sel_count, top_k, inputs_ready)
+        inputs_ready, single_launch: see rtp_layer_io."""
+        io = self._io(layer, mask, top_p, out, sel_count, top_k, inputs_ready, single_launch)
         _check(load().rtp_decode_step(self._h, layer_idx, ctypes.byref(io), _stream_ptr(stream)),
                "rtp_decode_step")
 

@@ -130,6 +130,16 @@ typedef struct {
                                 attention of a layer without retrieval heads stream their inputs
                                 while the previous launch drains; they still wait before
                                 writing anything the previous layer may read.                   */
+    int32_t single_launch;   /* 0 (default): the selection, attention and merge launches above.
+                                Nonzero: the whole layer in ONE cooperative launch of one CTA per
+                                SM (the pages' fused scoring + selection, extended through the
+                                gather): the retrieval slots' tokens are owned in 64-token tiles
+                                dealt round-robin to the CTAs, the selection stays in on-chip
+                                bit masks (no position list) and the split heads are merged after
+                                a grid barrier. Same selection and outputs as the default path.
+                                Needs B * Hkv <= 64 and B * nret * ceil(max_ctx / 64) <= 448 per
+                                SM, else RTP_ERR_UNSUPPORTED (nothing enqueued); inputs_ready is
+                                ignored (the launch always waits for the preceding one).          */
 } rtp_layer_io;
 
 /* Enqueues one layer of the decode step on `stream` (two kernels when the layer has retrieval

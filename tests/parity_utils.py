@@ -156,7 +156,7 @@ def make_handle(plan: W.Plan, **cfg_overrides) -> rtp.Handle:
 
 
 def run_layer(h: rtp.Handle, plan: W.Plan, li: W.LayerInputs, layer: int, top_p=None,
-              dense=False, top_k: int = 0):
+              dense=False, top_k: int = 0, single_launch: bool = False):
     B, Hq, Hkv = plan.batch, plan.num_q_heads, plan.num_kv_heads
     out = torch.full((B, Hq, 128), float("nan"), dtype=torch.float32, device=li.q.device)
     cnt = torch.full((B, Hkv), -1, dtype=torch.int32, device=li.q.device)
@@ -165,7 +165,7 @@ def run_layer(h: rtp.Handle, plan: W.Plan, li: W.LayerInputs, layer: int, top_p=
         h.dense_decode(L, out)
     else:
         h.decode_step(layer, L, plan.retrieval[layer], plan.top_p if top_p is None else top_p,
-                      out, cnt, top_k=top_k)
+                      out, cnt, top_k=top_k, single_launch=single_launch)
     torch.cuda.synchronize()
     return out, cnt
 
@@ -178,10 +178,11 @@ class LayerReport:
 
 
 def check_layer(h: rtp.Handle, plan: W.Plan, li: W.LayerInputs, layer: int, top_p=None,
-                heads=None, exact=True, top_k: int = 0) -> LayerReport:
+                heads=None, exact=True, top_k: int = 0,
+                single_launch: bool = False) -> LayerReport:
     """Run one layer on the GPU and compare every (or the given) head with the oracle."""
     p = plan.top_p if top_p is None else top_p
-    out, cnt = run_layer(h, plan, li, layer, p, top_k=top_k)
+    out, cnt = run_layer(h, plan, li, layer, p, top_k=top_k, single_launch=single_launch)
     assert h.device_status() == 0
     G = plan.group
     rep = LayerReport()
