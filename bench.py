@@ -113,6 +113,27 @@ def step_bytes(plan, sel_counts) -> tuple[int, int, int]:
     return idx + att, att, idx
 
 
+def exact_top_p_counts(plan, layers, top_p: float) -> list[int]:
+    """Size of the exact (sort-based) top-p set of every retrieval head of the workload, for the
+    overshoot statistic of the histogram selection: scores 0.25 q_idx . k_idx in fp32, masses
+    exp(s - s_max), the shortest prefix of the descending order whose mass reaches p of the total
+    (cumulative sums in fp64). A measurement aid run with torch ops, not part of the path."""
+    import torch
+    out = []
+    for l, li in enumerate(layers):
+        for b in range(plan.batch):
+            N = int(plan.seq_lens[b])
+            for h in range(plan.num_kv_heads):
+                if not plan.retrieval[l, h]:
+                    continue
+                k = li.k_idx[b, h, :N].float()
+                s = (k @ li.q_idx[b, h].float()) * 0.25
+                w = torch.exp(s - s.max()).double()
+                c = torch.cumsum(torch.sort(w, descending=True).values, 0)
+                out.append(int(torch.searchsorted(c, top_p * c[-1]).item()) + 1)
+    return out
+
+
 def cpu_sample_layers(plan, per_kind: int = 2):
     """A bounded sample of the workload for the CPU oracle (about 10 s of fp64 work at 1M
     context): per_kind layers with a broad (diffuse or flat) retrieval query, with a
@@ -565,6 +586,9 @@ def main():
     eff_gbs = total_bytes / (ms * 1e-3) / 1e9
     n_sel = [int(s[b, k]) for l, s in enumerate(sel) for b in range(B) for k in range(Hkv)
              if plan.retrieval[l, k]]
+    n_exact = exact_top_p_counts(plan, layers, plan.top_p) if n_sel else []
+    over = [a - e for a, e in zip(n_sel, n_exact)]
+    over_rel = [a / e - 1.0 for a, e in zip(n_sel, n_exact)]
     line = {
         "metric": METRIC, "value": value, "unit": "steps/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
@@ -588,7 +612,10 @@ def main():
         "kernels": kern,
         "selection": {"retrieval_heads": len(n_sel),
                       "mean_selected": float(np.mean(n_sel)) if n_sel else 0.0,
-                      "max_selected": int(max(n_sel)) if n_sel else 0},
+                      "max_selected": int(max(n_sel)) if n_sel else 0,
+                      "mean_exact_top_p": float(np.mean(n_exact)) if n_exact else 0.0,
+                      "overshoot_tokens_mean": float(np.mean(over)) if over else 0.0,
+                      "overshoot_rel_mean": float(np.mean(over_rel)) if over_rel else 0.0},
         "p_sweep": p_sweep,
         "k_sweep": k_sweep,
         "chained": chained,
