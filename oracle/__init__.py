@@ -61,6 +61,10 @@ def lib():
         L.orc_exact_topk.argtypes = [_dp, ctypes.c_int64, ctypes.c_int64, _i64p, _i64p]
         L.orc_window_sink_set.argtypes = [ctypes.c_int64, ctypes.c_int64, ctypes.c_int64,
                                           _i64p, _i64p]
+        L.orc_prefill_rows.argtypes = [_u16p, _u16p, _u16p, ctypes.c_int64, _i64p,
+                                       ctypes.c_int64, ctypes.c_int, ctypes.c_int,
+                                       ctypes.c_int64, ctypes.c_int64, ctypes.c_double,
+                                       ctypes.c_int, _dp]
         L.orc_sparse_attention.argtypes = [_u16p, _u16p, _u16p, _i64p, ctypes.c_int64,
                                            ctypes.c_int, ctypes.c_int, ctypes.c_double, _dp]
         L.orc_decode_layer.argtypes = [ctypes.POINTER(_LayerCfg), ctypes.c_int, _u16p, _u16p,
@@ -220,6 +224,28 @@ def sparse_attention(q, k, v, idx, scale: float | None = None) -> np.ndarray:
                                       _ptr(v, ctypes.c_uint16), _ptr(idx, ctypes.c_int64),
                                       idx.size, G, D, float(scale), _ptr(o, ctypes.c_double)),
            "sparse_attention")
+    return o
+
+
+def prefill_rows(q_rows, k, v, rows, dense: bool, window: int = 8192, sinks: int = 4,
+                 scale: float | None = None, num_threads: int | None = None) -> np.ndarray:
+    """Prefill attention of the prompt positions `rows` for one query head (fp64): row i
+    attends over {0..i} (dense: a retrieval head) or {0..sinks-1} U {i+1-window..i} (a local
+    head). q_rows [len(rows), D] holds those rows' queries; k, v [n_tok, D]; bf16 bits."""
+    q = _u16(q_rows)
+    k = _u16(k)
+    v = _u16(v)
+    rows = np.ascontiguousarray(rows, dtype=np.int64)
+    n_rows, D = q.shape
+    assert rows.shape == (n_rows,) and k.shape[1] == D and v.shape == k.shape
+    if scale is None:
+        scale = 1.0 / np.sqrt(D)
+    o = np.empty((n_rows, D), np.float64)
+    _check(lib().orc_prefill_rows(_ptr(q, ctypes.c_uint16), _ptr(k, ctypes.c_uint16),
+                                  _ptr(v, ctypes.c_uint16), k.shape[0], _ptr(rows, ctypes.c_int64),
+                                  n_rows, D, 1 if dense else 0, int(window), int(sinks),
+                                  float(scale), int(num_threads or 0), _ptr(o, ctypes.c_double)),
+           "prefill_rows")
     return o
 
 

@@ -37,7 +37,10 @@
  *     "洞察 3: 动态 Top-P 选择", top-2k / 4k / 16k): b* is the highest b whose suffix COUNT
  *     N_b = #{n : bin(n) >= b} reaches k (b* = 0, every token, when k >= n_tok);
  *   - a local head attends over {0..sinks-1} U {N-window..N-1} (set union, positions
- *     clipped to [0, N)); the cache already holds the current token at position N-1.
+ *     clipped to [0, N)); the cache already holds the current token at position N-1;
+ *   - prefill ([P3] Methodology 1: retrieval heads keep the full KV cache during prefill,
+ *     local heads the sliding window with sinks): prompt position i attends causally over the
+ *     key set a decode step of i + 1 tokens would use, dense for a retrieval head.
  *
  * All arithmetic is fp64 over the exact stored bf16 / fp16 values. Nothing is blocked,
  * fused or reordered beyond what the definitions above state.
@@ -427,6 +430,58 @@ int orc_sparse_attention(const uint16_t *q, const uint16_t *k, const uint16_t *v
     }
     free(x); free(qd);
     return ORC_OK;
+}
+
+/* ---- prefill: attention of every prompt position [P3 Methodology 1] --------------------- */
+
+/*
+ * Row i (0 <= i < n_tok) of the prompt attends over the key set of a context of i + 1 tokens:
+ * all of it, {0..i}, for a retrieval head (retrieval heads keep the full KV cache during
+ * prefill), and {0..sinks-1} U {i+1-window .. i} for a local head (sliding window with
+ * attention sinks). q holds the query rows listed in rows[] ([n_rows][D]); k, v [n_tok][D];
+ * o [n_rows][D]. One query head at a time (G = 1).
+ */
+int orc_prefill_rows(const uint16_t *q, const uint16_t *k, const uint16_t *v, int64_t n_tok,
+                     const int64_t *rows, int64_t n_rows, int D, int dense, int64_t window,
+                     int64_t sinks, double scale, int num_threads, double *o)
+{
+    if (!q || !k || !v || !rows || !o || n_tok <= 0 || n_rows < 0 || D <= 0)
+        return ORC_ERR_ARG;
+    for (int64_t r = 0; r < n_rows; r++)
+        if (rows[r] < 0 || rows[r] >= n_tok)
+            return ORC_ERR_ARG;
+    int err = ORC_OK;
+#ifdef _OPENMP
+#pragma omp parallel for schedule(dynamic, 1) num_threads(num_threads > 0 ? num_threads : omp_get_max_threads())
+#else
+    (void)num_threads;
+#endif
+    for (int64_t r = 0; r < n_rows; r++) {
+        const int64_t i = rows[r];
+        int64_t *idx = (int64_t *)malloc(sizeof(int64_t) * (size_t)(i + 1));
+        int64_t n = 0;
+        int rc = idx ? ORC_OK : ORC_ERR_NOMEM;
+        if (rc == ORC_OK) {
+            if (dense) {
+                for (int64_t j = 0; j <= i; j++)
+                    idx[j] = j;
+                n = i + 1;
+            } else {
+                rc = orc_window_sink_set(i + 1, window, sinks, idx, &n);
+            }
+        }
+        if (rc == ORC_OK)
+            rc = orc_sparse_attention(q + r * (int64_t)D, k, v, idx, n, 1, D, scale,
+                                      o + r * (int64_t)D);
+        free(idx);
+        if (rc != ORC_OK) {
+#ifdef _OPENMP
+#pragma omp critical
+#endif
+            err = rc;
+        }
+    }
+    return err;
 }
 
 /* ---- one layer of the decode step, every (batch, KV head) ------------------------------ */

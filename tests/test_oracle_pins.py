@@ -493,3 +493,62 @@ def test_layer_hist_contains_exact(orc):
     _, n_hist = orc.decode_layer(**io, top_p=0.9)
     _, n_exact = orc.decode_layer(**io, top_p=0.9, mode=orc.MODE_EXACT)
     assert n_exact[0, 0] <= n_hist[0, 0] < 20000
+
+
+# ---- prefill rows (every prompt position: causal; window + sinks for local heads) ---------
+
+def _prefill_masked_softmax(qv, kv, vv, dense, window, sinks):
+    """The whole T x T score matrix with a boolean mask, numpy softmax: a formulation of the
+    prefill rows independent of the oracle's per-row token sets."""
+    T, D = qv.shape
+    i = np.arange(T)[:, None]
+    j = np.arange(T)[None, :]
+    ok = j <= i
+    if not dense:
+        ok &= (j < sinks) | (j > i - window)
+    logits = np.where(ok, qv @ kv.T / math.sqrt(D), -np.inf)
+    return scipy.special.softmax(logits, axis=1) @ vv
+
+
+@pytest.mark.parametrize("dense,window,sinks", [(True, 8192, 4), (False, 7, 2), (False, 5, 0),
+                                                (False, 1, 3)])
+def test_prefill_rows_match_masked_matrix_softmax(orc, dense, window, sinks):
+    rng = np.random.default_rng(31)
+    T, D = 40, 128
+    qb, qv = _rand_bf16(rng, (T, D))
+    kb, kv = _rand_bf16(rng, (T, D))
+    vb, vv = _rand_bf16(rng, (T, D))
+    rows = np.arange(T)
+    o = orc.prefill_rows(qb, kb, vb, rows, dense, window, sinks)
+    ref = _prefill_masked_softmax(qv, kv, vv, dense, window, sinks)
+    assert np.allclose(o, ref, rtol=1e-12, atol=1e-13)
+
+
+def test_prefill_row_zero_and_zero_queries(orc):
+    rng = np.random.default_rng(32)
+    T, D = 25, 128
+    kb, _ = _rand_bf16(rng, (T, D))
+    vb, vv = _rand_bf16(rng, (T, D))
+    qb, _ = _rand_bf16(rng, (T, D), 3.0)
+    for dense in (True, False):
+        o0 = orc.prefill_rows(qb[:1], kb, vb, [0], dense, 6, 2)
+        assert np.array_equal(o0[0], vv[0])  # one key: the value row itself
+    zb = _bf16_bits(np.zeros((T, D)))
+    rows = np.arange(T)
+    od = orc.prefill_rows(zb, kb, vb, rows, True)
+    ol = orc.prefill_rows(zb, kb, vb, rows, False, 6, 2)
+    for i in range(T):  # a zero query weighs its keys equally: the mean of their values
+        assert np.allclose(od[i], vv[: i + 1].mean(0), rtol=1e-13, atol=1e-14)
+        keys = sorted(set(range(min(2, i + 1))) | set(range(max(0, i - 5), i + 1)))
+        assert np.allclose(ol[i], vv[keys].mean(0), rtol=1e-13, atol=1e-14)
+
+
+def test_prefill_window_covering_the_prompt_is_causal_dense(orc):
+    rng = np.random.default_rng(33)
+    T, D = 30, 128
+    qb, _ = _rand_bf16(rng, (T, D))
+    kb, _ = _rand_bf16(rng, (T, D))
+    vb, _ = _rand_bf16(rng, (T, D))
+    rows = np.arange(T)
+    assert np.array_equal(orc.prefill_rows(qb, kb, vb, rows, False, T, 4),
+                          orc.prefill_rows(qb, kb, vb, rows, True))
