@@ -212,7 +212,8 @@ RTP_API rtp_status rtp_get_threshold(rtp_handle *h, int b, int kvh, int *bstar, 
  * launches on this handle is bracketed by two CUDA events recorded on the launch stream (the
  * events are created here, so the decode calls still allocate nothing). Do not enable it while
  * capturing a CUDA graph. Kernel classes: 0 selection (indexer score, histogram top-p,
- * compaction), 1 attention, 2 merge of split heads' partials; 3 is reserved (always 0). The event pool holds 1024
+ * compaction), 1 attention, 2 merge of split heads' partials, 3 the single-launch layer
+ * (rtp_layer_io.single_launch). The event pool holds 1024
  * launches; rtp_profile_read empties it. Errors: RTP_ERR_CUDA if the events cannot be created. */
 RTP_API rtp_status rtp_profile_enable(rtp_handle *h, int enable);
 
