@@ -35,7 +35,7 @@ constexpr int kWarpStage = 2 * kTile * kRowBytes;          // 16 K rows then 16 
 constexpr int kOPitch = kHeadDim + 4;                      // padded row of the merge buffer
 constexpr int kCombFloats = kMaxGroup * kOPitch + kWarps * kMaxGroup * 2 + kMaxGroup * 2;
 constexpr int kMergeRows = kMergeThreads / 8;              // pieces a merge pass loads at once
-constexpr int kMergeRegs = 8;                              // passes kept in registers
+constexpr int kMergeRegs = 20;                             // passes kept in registers (320 pieces)
 
 // Shared memory: per-warp stages, the warp-merge buffer, then the head tables sized by the
 // layer (B * Hkv + 1 offsets, B lengths).

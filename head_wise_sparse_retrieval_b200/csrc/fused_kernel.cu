@@ -79,16 +79,6 @@ __device__ __forceinline__ int window_pos(int r, int N, int W, int S) {
   return (N <= W + S) ? r : (r < S ? r : N - W + (r - S));
 }
 
-// Order-preserving map of a float to an unsigned key (larger float, larger key; 0 is below
-// every key of a float, so 0 means "none").
-__device__ __forceinline__ unsigned float_key(float x) {
-  const unsigned u = __float_as_uint(x);
-  return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
-}
-__device__ __forceinline__ float key_float(unsigned k) {
-  return __uint_as_float((k & 0x80000000u) ? (k & 0x7FFFFFFFu) : ~k);
-}
-
 // Position of the k-th (0-based) set bit of x, k < popc(x): halving the window by popcounts.
 __device__ __forceinline__ int nth_set32(unsigned x, int k) {
   int pos = 0;

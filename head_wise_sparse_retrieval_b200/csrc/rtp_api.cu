@@ -267,6 +267,7 @@ rtp_status enqueue_layer(rtp_handle* h, const LayerArgs& a0, cudaStream_t s, int
     x.hist_cnt = h->hist_cnt;
     x.wait_ns = wait_ns;
     x.withhold_cta = withhold_cta;
+    x.smax_key = reinterpret_cast<unsigned*>(h->ws.cta_max);
     // the ranges are at most ceil(B * nret * max_ctx / grid) tokens: on chip when that fits
     const long long worst = (long long)a0.B * a0.nret * a0.max_ctx;
     const bool fits = (worst + h->select_grid - 1) / h->select_grid <= kScoreCap;
@@ -759,6 +760,8 @@ rtp_status rtp_get_device_status(rtp_handle* h, uint32_t* code) {
   // a barrier that timed out leaves its counter mid-count: start the next launch from zero
   if (e == cudaSuccess && (*code & kDevWaitTimeout)) {
     e = cudaMemset(h->ws.grid_bar, 0, (kFusedBarWord + 1) * 4);
+    if (e == cudaSuccess)  // a stopped selection may leave maxima behind
+      e = cudaMemset(h->ws.cta_max, 0, (size_t)h->cfg.batch * h->cfg.num_kv_heads * 4);
     if (e == cudaSuccess && h->fused_ok)  // a stopped single launch may leave maxima behind
       e = cudaMemset(h->fx.smax_key, 0, (size_t)h->cfg.batch * h->cfg.num_kv_heads * 4);
   }

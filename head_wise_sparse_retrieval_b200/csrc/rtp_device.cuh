@@ -100,6 +100,16 @@ __device__ inline void grid_barrier(unsigned* bar, unsigned* status, int* aborte
   __syncthreads();
 }
 
+// Order-preserving map of a float to an unsigned key (larger float, larger key; 0 is below
+// every key of a float, so 0 means "none").
+__device__ __forceinline__ unsigned float_key(float x) {
+  const unsigned u = __float_as_uint(x);
+  return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+__device__ __forceinline__ float key_float(unsigned k) {
+  return __uint_as_float((k & 0x80000000u) ? (k & 0x7FFFFFFFu) : ~k);
+}
+
 // ---- shared memory and asynchronous copies -----------------------------------------------
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {

@@ -14,7 +14,8 @@
 // grid barriers (bounded waits):
 //   1. scores: a lane pair reads a token's 32 bytes with two 16-byte loads (double-buffered),
 //      the scaled fp32 score is kept, and each CTA records the max of each slot it scores;
-//   2. histogram: s_max of a slot = max of its CTAs' maxima; every score is binned relative
+//   2. histogram: s_max of a slot = the atomic max of its CTAs' maxima (order-preserving
+//      integer keys, cleared after the second barrier); every score is binned relative
 //      to s_max and exp(s - s_max) is added in 2^-40 fixed point to per-warp shared bins
 //      (32-bit words, exact integer sums whatever the order). The CTA adds its masses to one
 //      of kHistCopies copies of the slot's global histogram (integer atomics, spread over the
@@ -281,7 +282,7 @@ __device__ __forceinline__ void select_body(const LayerArgs& a, const Workspace&
         for (int u = 0; u < kUnroll; ++u) kv[u] = nx[u];
       }
       mx = block_max(mx, redf);
-      if (tid == 0) w.cta_max[(size_t)s * gridDim.x + blockIdx.x] = mx;
+      if (tid == 0) atomicMax(x.smax_key + s, float_key(mx));
     }
   }
   grid_barrier(w.grid_bar, w.status, &aborted, x.wait_ns, x.withhold_cta);
@@ -293,16 +294,15 @@ __device__ __forceinline__ void select_body(const LayerArgs& a, const Workspace&
       const int n0 = (int)(t - soff[s]);
       const int n1 = (int)(min(t1, soff[s + 1]) - soff[s]);
       t = soff[s] + n1;
-      const long long c0 = cta_of(soff[s], T, P), c1 = cta_of(soff[s + 1] - 1, T, P);
-      float m = -INFINITY;  // s_max of the slot: max over the CTAs that scored it
-      for (long long c = c0 + tid; c <= c1; c += kSelThreads)
-        m = fmaxf(m, __ldcg(w.cta_max + (size_t)s * gridDim.x + c));
+      const long long c0 = cta_of(soff[s], T, P);
+      // s_max of the slot: the atomic max over the CTAs that scored it
+      const float s_max = key_float(__ldcg(x.smax_key + s));
       for (int i = tid; i < kWarpsSel * kBins; i += kSelThreads) {
         (&wlo[0][0])[i] = 0u;
         (&whi[0][0])[i] = 0u;
       }
       cnt[tid] = 0u;
-      const float s_max = block_max(m, redf);  // its barriers also order the zero fill
+      __syncthreads();  // the zero fill comes before the adds
       const int copy = (int)(blockIdx.x % kHistCopies);
       // bits 0..19 and 20..40 of the 2^-40 weights go to separate 32-bit words, so that no add
       // needs the old value: a warp adds at most kScoreCap / 8 tokens to a bin before the flush
@@ -344,6 +344,8 @@ __device__ __forceinline__ void select_body(const LayerArgs& a, const Workspace&
     }
   }
   grid_barrier(w.grid_bar, w.status, &aborted, x.wait_ns, -1);
+  if (blockIdx.x == 0 && !aborted)  // every CTA read the maxima before this barrier
+    for (int s = tid; s < S; s += kSelThreads) x.smax_key[s] = 0u;
 
   // ---- phase 3: b*, offsets and the dense selected list -----------------------------------
   if (active) {
