@@ -123,7 +123,7 @@ WsPlan plan_workspace(const rtp_config* c, int attend_grid, int select_grid, int
   const bool fused = slots <= (size_t)kFusedMaxHeads;
   const size_t sizes[] = {
       slots * nmax * 4,                      // 0 scores
-      slots * (size_t)select_grid * 4,       // 1 cta_max
+      slots * 4,                             // 1 smax_key
       (size_t)kHistCopies * slots * kBins * 8,  // 2 hist
       slots * 4,                             // 3 s_max
       slots * 4,                             // 4 bstar
@@ -267,7 +267,6 @@ rtp_status enqueue_layer(rtp_handle* h, const LayerArgs& a0, cudaStream_t s, int
     x.hist_cnt = h->hist_cnt;
     x.wait_ns = wait_ns;
     x.withhold_cta = withhold_cta;
-    x.smax_key = reinterpret_cast<unsigned*>(h->ws.cta_max);
     // the ranges are at most ceil(B * nret * max_ctx / grid) tokens: on chip when that fits
     const long long worst = (long long)a0.B * a0.nret * a0.max_ctx;
     const bool fits = (worst + h->select_grid - 1) / h->select_grid <= kScoreCap;
@@ -401,7 +400,7 @@ rtp_status rtp_create(const rtp_config* cfg, int device, rtp_handle** out) {
   char* base = static_cast<char*>(h->ws_mem);
   Workspace& w = h->ws;
   w.scores = reinterpret_cast<float*>(base + p.off[0]);
-  w.cta_max = reinterpret_cast<float*>(base + p.off[1]);
+  w.smax_key = reinterpret_cast<unsigned*>(base + p.off[1]);
   w.hist = reinterpret_cast<unsigned long long*>(base + p.off[2]);
   w.s_max = reinterpret_cast<float*>(base + p.off[3]);
   w.bstar = reinterpret_cast<int*>(base + p.off[4]);
@@ -761,7 +760,7 @@ rtp_status rtp_get_device_status(rtp_handle* h, uint32_t* code) {
   if (e == cudaSuccess && (*code & kDevWaitTimeout)) {
     e = cudaMemset(h->ws.grid_bar, 0, (kFusedBarWord + 1) * 4);
     if (e == cudaSuccess)  // a stopped selection may leave maxima behind
-      e = cudaMemset(h->ws.cta_max, 0, (size_t)h->cfg.batch * h->cfg.num_kv_heads * 4);
+      e = cudaMemset(h->ws.smax_key, 0, (size_t)h->cfg.batch * h->cfg.num_kv_heads * 4);
     if (e == cudaSuccess && h->fused_ok)  // a stopped single launch may leave maxima behind
       e = cudaMemset(h->fx.smax_key, 0, (size_t)h->cfg.batch * h->cfg.num_kv_heads * 4);
   }

@@ -15,8 +15,8 @@ constexpr int kMaxKvHeads = 256;
 struct Workspace {
   float* scores;                  // [slots][ld]             scaled indexer scores (spill)
   unsigned char* bins;            // [slots][ld]             their histogram bins (spill)
-  float* cta_max;                 // [slots][select_ctas]    (the selection uses the first
-                                  // slots words as SelectArgs::smax_key)
+  unsigned* smax_key;             // [slots]                 atomic max of the CTAs' maxima
+                                  //                         (float_key); 0 between launches
   unsigned long long* hist;       // [kHistCopies][slots][256] fixed-point (2^-40) bin masses
   float* s_max;                   // [slots]
   int* bstar;                     // [slots]
@@ -38,8 +38,6 @@ struct SelectArgs {
   unsigned* hist_cnt;             // [kHistCopies][slots][256] tokens per bin (top-k only)
   unsigned long long wait_ns;     // limit of every grid-barrier wait
   int withhold_cta;               // self-test: CTA that skips its first arrival, else -1
-  unsigned* smax_key;             // [slots] atomic max of the CTAs' maxima (order-preserving
-                                  // keys, float_key); 0 between launches
 };
 
 struct LayerArgs {

@@ -282,7 +282,7 @@ __device__ __forceinline__ void select_body(const LayerArgs& a, const Workspace&
         for (int u = 0; u < kUnroll; ++u) kv[u] = nx[u];
       }
       mx = block_max(mx, redf);
-      if (tid == 0) atomicMax(x.smax_key + s, float_key(mx));
+      if (tid == 0) atomicMax(w.smax_key + s, float_key(mx));
     }
   }
   grid_barrier(w.grid_bar, w.status, &aborted, x.wait_ns, x.withhold_cta);
@@ -296,7 +296,7 @@ __device__ __forceinline__ void select_body(const LayerArgs& a, const Workspace&
       t = soff[s] + n1;
       const long long c0 = cta_of(soff[s], T, P);
       // s_max of the slot: the atomic max over the CTAs that scored it
-      const float s_max = key_float(__ldcg(x.smax_key + s));
+      const float s_max = key_float(__ldcg(w.smax_key + s));
       for (int i = tid; i < kWarpsSel * kBins; i += kSelThreads) {
         (&wlo[0][0])[i] = 0u;
         (&whi[0][0])[i] = 0u;
@@ -345,7 +345,7 @@ __device__ __forceinline__ void select_body(const LayerArgs& a, const Workspace&
   }
   grid_barrier(w.grid_bar, w.status, &aborted, x.wait_ns, -1);
   if (blockIdx.x == 0 && !aborted)  // every CTA read the maxima before this barrier
-    for (int s = tid; s < S; s += kSelThreads) x.smax_key[s] = 0u;
+    for (int s = tid; s < S; s += kSelThreads) w.smax_key[s] = 0u;
 
   // ---- phase 3: b*, offsets and the dense selected list -----------------------------------
   if (active) {
