@@ -396,3 +396,20 @@ def test_long_configs_sampled_layers(name):
             check_layer(h, p, li, l, exact=False)
             del li
             torch.cuda.empty_cache()
+
+
+def test_maximum_head_count():
+    """B * Hkv = 1024 heads (the largest layer the library takes), 256 retrieval slots and
+    32 768 merge units, ragged contexts from 1 to 300 tokens; sampled heads against the
+    oracle."""
+    B, Hkv, G = 64, 16, 8
+    rng = np.random.default_rng(5)
+    seqs = [int(x) for x in rng.integers(1, 301, B)]
+    ret = [1 if k % 4 == 0 else 0 for k in range(Hkv)]
+    kinds = [[(W.KIND_DIFFUSE if (b + k) % 2 else W.KIND_CONC) if ret[k] else W.KIND_LOCAL
+              for k in range(Hkv)] for b in range(B)]
+    needles = [[2 if kinds[b][k] == W.KIND_CONC else 0 for k in range(Hkv)] for b in range(B)]
+    p = W.custom(batch=B, num_q_heads=Hkv * G, num_kv_heads=Hkv, seq_lens=seqs, max_ctx=300,
+                 retrieval=ret, kinds=kinds, n_needles=needles, seed=17)
+    heads = [(b, k) for b in (0, 1, 31, 62, 63) for k in (0, 3, 4, 12, 15)]
+    _run(p, heads=heads, exact=False)

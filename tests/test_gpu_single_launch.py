@@ -212,3 +212,17 @@ def test_ctx_1m_sampled_layers():
             check_layer(h, p, li, l, exact=False, single_launch=True)
             del li
             torch.cuda.empty_cache()
+
+
+def test_largest_single_launch_layer():
+    """B * Hkv = 64, the largest layer the single-launch tables take, with ragged contexts."""
+    B, Hkv = 16, 4
+    seqs = [1 + 997 * b for b in range(B)]
+    kinds = [[W.KIND_DIFFUSE, W.KIND_LOCAL, W.KIND_CONC, W.KIND_FLAT] for _ in range(B)]
+    p = W.custom(batch=B, num_q_heads=32, num_kv_heads=Hkv, seq_lens=seqs, max_ctx=max(seqs),
+                 retrieval=[1, 0, 1, 1], kinds=kinds, n_needles=[[0, 0, 3, 0]] * B, seed=23)
+    li = W.make_layer(p, 0, DEV)
+    heads = [(b, k) for b in (0, 1, 7, 15) for k in range(Hkv)]
+    with make_handle(p) as h:
+        check_layer(h, p, li, 0, heads=heads, exact=False, single_launch=True)
+    _same_selection_as_three_launches(p)
