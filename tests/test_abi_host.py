@@ -74,3 +74,12 @@ def test_calls_on_null_handle_are_rejected(rtp_lib):
         rtp_lib.RTP_ERR_INVALID_ARG
     assert L.rtp_destroy(None) == rtp_lib.RTP_OK
     assert L.rtp_status_string(3) == b"RTP_ERR_OOM"
+
+
+def test_workspace_holds_single_launch_buffers_only_within_its_limits(rtp_lib):
+    """The single-launch layer's pieces (one per CTA and head, 4160 bytes each), masks and keys
+    are planned for B * Hkv <= 64 only: 68 heads need less workspace than 64."""
+    ws = lambda B: rtp_lib.workspace_bytes(rtp_lib.default_config(1, B, 32, 4, 4096))
+    within, beyond = ws(16), ws(17)          # 64 heads, then 68 heads
+    assert 0 < beyond < within
+    assert within - beyond > 16 << 20        # 64 x (one piece per SM) x 4160 B alone is ~39 MB
