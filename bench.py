@@ -603,6 +603,8 @@ def main():
                    "timing": "CUDA graph of all layers, CUDA events on the launch stream"},
         "effective_gbs": eff_gbs,
         "roofline_frac_step": eff_gbs / hbm,
+        # the same against the data-sheet HBM3e figure of a B200 (8 TB/s), for context
+        "roofline_frac_step_nominal_8tbs": eff_gbs / 8000.0,
         "algorithmic_bytes_per_step": total_bytes,
         "bytes_breakdown": {"indexer": idx_bytes, "attend_kv": attend_bytes},
         "roofline": {"bound": "hbm", "kernel": "attend_kernel", "achieved": att_gbs,
