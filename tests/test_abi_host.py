@@ -83,3 +83,19 @@ def test_workspace_holds_single_launch_buffers_only_within_its_limits(rtp_lib):
     within, beyond = ws(16), ws(17)          # 64 heads, then 68 heads
     assert 0 < beyond < within
     assert within - beyond > 16 << 20        # 64 x (one piece per SM) x 4160 B alone is ~39 MB
+
+
+@pytest.mark.parametrize("compiler,std,lang", [("gcc", "-std=c99", "c"), ("g++", "-std=c++17", "c++")])
+def test_header_compiles_as_c_and_cpp(tmp_path, compiler, std, lang):
+    """include/rtp.h is a plain C header (no torch, no CUDA types in the signatures)."""
+    import shutil
+    import subprocess
+    if shutil.which(compiler) is None:
+        pytest.skip(f"{compiler} not installed")
+    src = tmp_path / "use_rtp.c"
+    src.write_text('#include "rtp.h"\nint main(void) { rtp_layer_io io; io.single_launch = 1;'
+                   ' (void)io; return rtp_status_string(RTP_OK) ? 0 : 1; }\n')
+    r = subprocess.run([compiler, std, "-Wall", "-Wextra", "-Werror", "-fsyntax-only", "-x", lang,
+                        "-I", os.path.join(ROOT, "include"), str(src)],
+                       capture_output=True, text=True)
+    assert r.returncode == 0, r.stderr
