@@ -99,8 +99,10 @@ extern "C" rtp_status rtp_window_attention_noalloc(const rtp_noalloc_params* p, 
 
   const int nheads = p->batch * p->num_kv_heads;
   const size_t smem = attend_smem_bytes(nheads, p->batch);
-  // the dynamic shared memory limit is a per-kernel setting; raising it is not an allocation
-  e = cudaFuncSetAttribute(attend_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  // the dynamic shared memory limit is a per-kernel setting shared with every handle; it is
+  // only ever raised (a handle created earlier for a larger layer keeps its size), and raising
+  // it is not an allocation
+  e = raise_smem_limit((const void*)attend_kernel, smem);
   if (e != cudaSuccess) return na_fail(RTP_ERR_CUDA, "cannot set the kernel's shared memory");
 
   LayerArgs a;

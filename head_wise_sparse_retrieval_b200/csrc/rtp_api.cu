@@ -3,6 +3,7 @@
 #include <cstdarg>
 #include <cstdio>
 #include <cstring>
+#include <mutex>
 #include <vector>
 
 #include "rtp.h"
@@ -96,8 +97,9 @@ rtp_status check_config(const rtp_config* c) {
   if (c->head_dim != kHeadDim) return fail(RTP_ERR_UNSUPPORTED, "head_dim must be 128");
   if (c->idx_dim != kIdxDim) return fail(RTP_ERR_UNSUPPORTED, "idx_dim must be 16");
   if (c->num_bins != kBins) return fail(RTP_ERR_UNSUPPORTED, "num_bins must be 256");
-  if (c->max_ctx < 1 || c->max_ctx > (1 << 28))
-    return fail(RTP_ERR_INVALID_ARG, "max_ctx must be in [1, 2^28]");
+  if (c->max_ctx < 1 || c->max_ctx > kMaxCtx)
+    return fail(RTP_ERR_INVALID_ARG,
+                "max_ctx must be in [1, 2^24 - 1] (the 64-bit fixed-point mass sums)");
   if (c->window < 1) return fail(RTP_ERR_INVALID_ARG, "window must be >= 1");
   if (c->sinks < 0) return fail(RTP_ERR_INVALID_ARG, "sinks must be >= 0");
   if (c->window > (1 << 28) || c->sinks > (1 << 28))
@@ -301,6 +303,16 @@ struct DeviceGuard {
 namespace rtp {
 // Records the reason returned by rtp_last_error on this thread (used by noalloc.cu).
 void set_last_error(const char* msg) { snprintf(g_err, sizeof g_err, "%s", msg); }
+
+cudaError_t raise_smem_limit(const void* kernel, size_t bytes) {
+  static std::mutex mu;  // the read and the raise are one step for concurrent callers
+  std::lock_guard<std::mutex> lock(mu);
+  cudaFuncAttributes fa;
+  cudaError_t e = cudaFuncGetAttributes(&fa, kernel);  // the current device's setting
+  if (e != cudaSuccess) return e;
+  if (bytes <= (size_t)fa.maxDynamicSharedSizeBytes) return cudaSuccess;
+  return cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
+}
 }  // namespace rtp
 
 extern "C" {
@@ -352,11 +364,8 @@ rtp_status rtp_create(const rtp_config* cfg, int device, rtp_handle** out) {
   if (h->attend_grid > kMaxPieces) h->attend_grid = kMaxPieces;
 
   h->select_smem = select_smem_bytes(cfg->batch * cfg->num_kv_heads);
-  e = cudaFuncSetAttribute(select_kernel_onchip, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           (int)h->select_smem);
-  if (e == cudaSuccess)
-    e = cudaFuncSetAttribute(select_kernel_spill, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             (int)h->select_smem);
+  e = raise_smem_limit((const void*)select_kernel_onchip, h->select_smem);
+  if (e == cudaSuccess) e = raise_smem_limit((const void*)select_kernel_spill, h->select_smem);
   int sel_per_sm = 0, sel_per_sm_spill = 0;
   if (e == cudaSuccess)
     e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&sel_per_sm, select_kernel_onchip,
@@ -436,8 +445,7 @@ rtp_status rtp_create(const rtp_config* cfg, int device, rtp_handle** out) {
     delete h;
     return fail(RTP_ERR_UNSUPPORTED, "max_ctx too large for the attention kernel's shared memory");
   }
-  e = cudaFuncSetAttribute(attend_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           (int)h->attend_smem);
+  e = raise_smem_limit((const void*)attend_kernel, h->attend_smem);
   if (e == cudaSuccess)
     e = cudaFuncSetAttribute(attend_kernel, cudaFuncAttributePreferredSharedMemoryCarveout, 100);
   if (e != cudaSuccess) {
@@ -449,8 +457,7 @@ rtp_status rtp_create(const rtp_config* cfg, int device, rtp_handle** out) {
       fused_smem_bytes() <= (size_t)max_optin) {
     h->fused_smem = fused_smem_bytes();
     int per_sm = 0;
-    e = cudaFuncSetAttribute(fused_layer_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             (int)h->fused_smem);
+    e = raise_smem_limit((const void*)fused_layer_kernel, h->fused_smem);
     if (e == cudaSuccess)
       e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, fused_layer_kernel,
                                                         kFusedThreads, h->fused_smem);

@@ -10,6 +10,11 @@ namespace rtp {
 
 constexpr int kMaxKvHeads = 256;
 
+// Largest cache a handle takes. The selection sums each token's mass exp(s - s_max) in (0, 1]
+// as an integer of 2^-40 units (at most 2^40 per token) into 64-bit bins and a 64-bit total,
+// so N tokens must satisfy N * 2^40 < 2^64: N <= 2^24 - 1.
+constexpr int kMaxCtx = (1 << 24) - 1;
+
 // Device workspace owned by a handle. Slot = b * nret + j for the j-th retrieval KV head of
 // the current layer (the workspace is sized for nret = Hkv).
 struct Workspace {
@@ -128,5 +133,11 @@ __host__ __device__ inline int merge_units(int nheads, int G) { return nheads * 
 
 size_t attend_smem_bytes(int nheads, int batch);
 void set_last_error(const char* msg);  // the reason rtp_last_error reports on this thread
+
+// Raises a kernel's cudaFuncAttributeMaxDynamicSharedMemorySize on the current device to at
+// least `bytes`, never lowering it. The attribute is one setting per kernel and device for the
+// whole process, shared by every handle and by the no-allocation entry point: lowering it for a
+// smaller layer would make a larger handle's later launches fail. Thread-safe.
+cudaError_t raise_smem_limit(const void* kernel, size_t bytes);
 
 }  // namespace rtp

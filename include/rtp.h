@@ -77,7 +77,8 @@ typedef struct {
     int num_kv_heads;  /* Hkv, 1 .. 256; G = Hq / Hkv must be 1 .. 8                           */
     int head_dim;      /* D, 128 only                                                          */
     int idx_dim;       /* r, 16 only                                                           */
-    int max_ctx;       /* cache capacity per (b, KV head), 1 .. 2^28                           */
+    int max_ctx;       /* cache capacity per (b, KV head), 1 .. 2^24 - 1 (16 777 215): the
+                          selection sums token masses as 64-bit integers of 2^-40 units    */
     int window;        /* local-head sliding window, >= 1 (8192)                               */
     int sinks;         /* local-head sink tokens, >= 0 (4)                                     */
     int num_bins;      /* histogram bins, 256 only                                             */

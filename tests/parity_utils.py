@@ -8,7 +8,18 @@ Tolerances (fixed by the method's stated bar):
     a bin edge (they may fall on either side in fp32); a different threshold bin is accepted
     only when the oracle's suffix mass at the disputed boundary is within 1e-6 * C_0 of
     p * C_0 ("threshold-ambiguous");
-  * outputs: max |gpu - oracle| <= 1e-2 and mean |gpu - oracle| <= 1e-3 per layer.
+  * outputs, absolute (the method's stated bar): max |gpu - oracle| <= 1e-2 and
+    mean |gpu - oracle| <= 1e-3 per head and per layer, against O1 over the oracle's set;
+  * outputs, relative (per head, G x 128 values): max |err| <= 1e-2 * max |ref| + 1e-6 and
+    mean |err| <= 1e-2 * mean |ref| + 1e-6, against O1 recomputed over the GPU's own set, so
+    that a broad head whose output is ~1e-3 in size cannot pass with a wrong or half-sized
+    result. The bound comes from the kernel's arithmetic: the softmax weights are rounded to
+    bf16 (relative error at most 2^-9, about uniform, so of standard deviation 2^-9/sqrt(3))
+    and the normaliser is summed from the same rounded weights, so the output is a convex
+    combination with perturbed weights: err = sum_n p_n d_n (v_n - o) / sum_n p_n. For the
+    random values of these workloads both err and o scale as sqrt(sum p_n^2) / sum p_n, and
+    their ratio is about 2^-9/sqrt(3) = 1.1e-3; 1e-2 leaves a margin of about 9x. A head
+    concentrated on a few tokens has |err| <= 2^-9 |v_a - v_b| with |o| of order one.
 """
 from __future__ import annotations
 
@@ -24,6 +35,8 @@ from head_wise_sparse_retrieval_b200 import workloads as W
 
 MAX_ABS = 1e-2
 MEAN_ABS = 1e-3
+REL = 1e-2
+REL_FLOOR = 1e-6
 EDGE_TOL = 1e-5
 AMBIG_TOL = 1e-6
 
@@ -143,12 +156,35 @@ def check_selection_topk(gpu_sel: np.ndarray, gpu_bstar: int, ho: HeadOracle,
                            gpu_bstar)
 
 
-def check_output(gpu: np.ndarray, ref: np.ndarray, what: str = ""):
-    err = np.abs(gpu.astype(np.float64) - ref)
+def check_output(gpu: np.ndarray, ref: np.ndarray, what: str = "",
+                 own: np.ndarray | None = None):
+    """One head's output ([G, 128]) against the oracle: the absolute bar against ref (O1 over
+    the oracle's set) and the relative bar against own (O1 over the GPU's set; ref when the
+    sets agree)."""
     assert np.isfinite(gpu).all(), f"{what}: non-finite output"
+    g = gpu.astype(np.float64)
+    err = np.abs(g - ref)
     mx, mean = float(err.max()), float(err.mean())
     assert mx <= MAX_ABS and mean <= MEAN_ABS, f"{what}: max-abs {mx:.3e}, mean-abs {mean:.3e}"
+    base = ref if own is None else own
+    rerr = np.abs(g - base)
+    rmx, rmean = float(rerr.max()), float(rerr.mean())
+    lim_mx = REL * float(np.abs(base).max()) + REL_FLOOR
+    lim_mean = REL * float(np.abs(base).mean()) + REL_FLOOR
+    assert rmx <= lim_mx and rmean <= lim_mean, (
+        f"{what}: relative bar: max |err| {rmx:.3e} > {lim_mx:.3e} or mean |err| {rmean:.3e} > "
+        f"{lim_mean:.3e} (max |ref| {float(np.abs(base).max()):.3e})")
     return mx, mean
+
+
+def own_set_output(li: W.LayerInputs, b: int, kvh: int, G: int, sel: np.ndarray) -> np.ndarray:
+    """O1 recomputed by the oracle over the positions the GPU selected (to tell kernel error
+    from a selection that differs at bin edges)."""
+    q = u16(li.q[b, kvh * G:(kvh + 1) * G])
+    rows = torch.as_tensor(np.asarray(sel, np.int64), device=li.k_cache.device)
+    k = u16(li.k_cache[b, kvh].index_select(0, rows))
+    v = u16(li.v_cache[b, kvh].index_select(0, rows))
+    return oracle.sparse_attention(q, k, v, np.arange(len(sel)), 1.0 / math.sqrt(128))
 
 
 def make_handle(plan: W.Plan, **cfg_overrides) -> rtp.Handle:
@@ -204,12 +240,17 @@ def check_layer(h: rtp.Handle, plan: W.Plan, li: W.LayerInputs, layer: int, top_
                 sr = check_selection(gsel, gb, ho, p, exact=exact)
             info["sel"] = sr
             assert cnt_h[b, kvh] == gsel.size
+            own = None
             if sr.edge_tokens == 0 and not sr.ambiguous:
                 assert gsel.size == ho.sel.size
+            else:  # the sets differ at bin edges: isolate the kernel's error on its own set
+                own = own_set_output(li, b, kvh, G, gsel)
+                info["own_set"] = True
         else:
             assert cnt_h[b, kvh] == ho.sel.size
+            own = None
         g = out_h[b, kvh * G:(kvh + 1) * G]
-        mx, mean = check_output(g, ho.out, f"layer {layer} b {b} kvh {kvh}")
+        mx, mean = check_output(g, ho.out, f"layer {layer} b {b} kvh {kvh}", own)
         errs.append(np.abs(g - ho.out))
         rep.heads.append(info)
     e = np.concatenate([x.ravel() for x in errs])

@@ -51,7 +51,7 @@ def test_workspace_is_linear_in_context(rtp_lib):
     ("head_dim", 64, 2), ("idx_dim", 32, 2), ("num_bins", 128, 2), ("num_q_heads", 36, 2),
     ("num_q_heads", 30, 1), ("max_ctx", 0, 1), ("window", 0, 1), ("sinks", -1, 1),
     ("idx_range", 0.0, 1), ("idx_scale", -1.0, 1), ("attn_scale", float("inf"), 1),
-    ("batch", 0, 1), ("num_layers", 0, 1),
+    ("batch", 0, 1), ("num_layers", 0, 1), ("max_ctx", 1 << 24, 1), ("max_ctx", 1 << 28, 1),
 ])
 def test_create_rejects_bad_config_before_touching_the_device(rtp_lib, field, value, status):
     c = rtp_lib.default_config(2, 1, 32, 4, 4096)
@@ -61,6 +61,21 @@ def test_create_rejects_bad_config_before_touching_the_device(rtp_lib, field, va
     assert st == status
     assert not h.value
     assert rtp_lib.load().rtp_last_error().decode()
+
+
+def test_max_ctx_stops_where_the_fixed_point_mass_sums_would_wrap(rtp_lib):
+    """Token masses in (0, 1] are summed as 64-bit integers of 2^-40 units: N tokens of mass 1
+    reach N * 2^40, which wraps at N = 2^24. The last context that cannot wrap is accepted, the
+    first one that can is refused."""
+    ok = rtp_lib.workspace_bytes(rtp_lib.default_config(1, 1, 8, 1, (1 << 24) - 1))
+    assert ok > 0
+    assert ((1 << 24) - 1) * (1 << 40) < 1 << 64 <= (1 << 24) * (1 << 40)
+    assert rtp_lib.workspace_bytes(rtp_lib.default_config(1, 1, 8, 1, 1 << 24)) == 0
+    c = rtp_lib.default_config(1, 1, 8, 1, 1 << 24)
+    h = ctypes.c_void_p()
+    assert rtp_lib.load().rtp_create(ctypes.byref(c), 0, ctypes.byref(h)) == \
+        rtp_lib.RTP_ERR_INVALID_ARG
+    assert "2^24" in rtp_lib.load().rtp_last_error().decode()
 
 
 def test_calls_on_null_handle_are_rejected(rtp_lib):
