@@ -191,6 +191,7 @@ __device__ __forceinline__ void select_body(const LayerArgs& a, const Workspace&
   __shared__ int bstar_s;
 
   __shared__ unsigned long long red64[kWarpsSel];
+  __shared__ unsigned long long bin0_mass;     // bin 0's fixed-point mass in the chunk
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int S = a.B * a.nret;
@@ -313,8 +314,14 @@ __device__ __forceinline__ void select_body(const LayerArgs& a, const Workspace&
             (&wlo[0][0])[i] = 0u;
             (&whi[0][0])[i] = 0u;
           }
-          __syncthreads();
         }
+        if (tid == 0) bin0_mass = 0ull;
+        __syncthreads();
+        // Bin 0 takes every score below the range: for a query with a few dominant tokens that
+        // is most of the slot, and shared atomics on that one bin would serialise the warp.
+        // Its tokens are summed in registers instead, then once per warp.
+        unsigned long long m0 = 0ull;
+        unsigned n0cnt = 0u;
 #pragma unroll 4
         for (int n = k0 + tid; n < k1; n += kSelThreads) {
           const float v = *sc.at(s, n);
@@ -322,12 +329,26 @@ __device__ __forceinline__ void select_body(const LayerArgs& a, const Workspace&
           *sc.bin_at(s, n) = (unsigned char)bin;
           const float wgt = expf(v - s_max);                          // in (0, 1]
           const unsigned long long fx = __float2ull_rn(wgt * 1099511627776.0f);  // * 2^40, exact
-          atomicAdd(&wlo[warp][bin], (uint32_t)fx & 0xFFFFFu);
-          atomicAdd(&whi[warp][bin], (uint32_t)(fx >> 20));
-          atomicAdd(&cnt[bin], 1u);
+          if (bin == 0) {
+            m0 += fx;
+            ++n0cnt;
+          } else {
+            atomicAdd(&wlo[warp][bin], (uint32_t)fx & 0xFFFFFu);
+            atomicAdd(&whi[warp][bin], (uint32_t)(fx >> 20));
+            atomicAdd(&cnt[bin], 1u);
+          }
+        }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) {
+          m0 += __shfl_xor_sync(0xffffffffu, m0, o);
+          n0cnt += __shfl_xor_sync(0xffffffffu, n0cnt, o);
+        }
+        if (lane == 0 && n0cnt) {
+          atomicAdd(&bin0_mass, m0);
+          atomicAdd(&cnt[0], n0cnt);
         }
         __syncthreads();
-        unsigned long long v = 0ull;
+        unsigned long long v = (tid == 0) ? bin0_mass : 0ull;
 #pragma unroll
         for (int k = 0; k < kWarpsSel; ++k)
           v += ((unsigned long long)whi[k][tid] << 20) + wlo[k][tid];
