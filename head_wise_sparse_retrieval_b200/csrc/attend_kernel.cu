@@ -62,6 +62,21 @@ __device__ __forceinline__ int window_pos(int r, int N, int W, int S) {
   return (N <= W + S) ? r : (r < S ? r : N - W + (r - S));
 }
 
+// Size of head hd's token set (retrieval: |S| from the selection, clamped to [1, N]; local:
+// the window set; dense: N), N = seq_lens[b] clamped to [1, max_ctx]. The attention split and
+// the merge both derive the pieces of a head from these sizes.
+__device__ __forceinline__ int head_len(const LayerArgs& a, const Workspace& w, int hd, int* N_out) {
+  const int b = hd / a.Hkv, kvh = hd - b * a.Hkv;
+  const bool ret = !a.dense && a.slot_of_kvh[kvh] >= 0;
+  const int n = a.seq_lens[b];  // both loads in flight together
+  const int ns = ret ? __ldcg(w.sel_total + b * a.nret + a.slot_of_kvh[kvh]) : 0;
+  const int N = n < 1 ? 1 : (n > a.max_ctx ? a.max_ctx : n);
+  if (N_out) *N_out = N;
+  if (a.dense) return N;
+  if (ret) return ns < 1 ? 1 : (ns > N ? N : ns);
+  return window_len(N, a.window, a.sinks);
+}
+
 // The segments of this CTA's range, head by head, in order.
 struct Walk {
   const long long* off;
@@ -205,20 +220,9 @@ __global__ void __launch_bounds__(kAttendThreads, kAttendCtasPerSm) attend_kerne
 
   // ---- the layer's heads and their token-set lengths --------------------------------------
   for (int hd = tid; hd < nheads; hd += kAttendThreads) {
-    const int b = hd / a.Hkv, kvh = hd - b * a.Hkv;
-    const bool ret = !a.dense && a.slot_of_kvh[kvh] >= 0;
-    const int n = a.seq_lens[b];  // both loads in flight together
-    const int ns = ret ? __ldcg(w.sel_total + b * a.nret + a.slot_of_kvh[kvh]) : 0;
-    const int N = n < 1 ? 1 : (n > a.max_ctx ? a.max_ctx : n);
-    if (kvh == 0) sSeq[b] = N;
-    int len;
-    if (a.dense) {
-      len = N;
-    } else if (ret) {
-      len = ns < 1 ? 1 : (ns > N ? N : ns);
-    } else {
-      len = window_len(N, a.window, a.sinks);
-    }
+    int N;
+    const int len = head_len(a, w, hd, &N);
+    if (hd % a.Hkv == 0) sSeq[hd / a.Hkv] = N;
     sOff[hd + 1] = len;
   }
   __syncthreads();
@@ -528,12 +532,45 @@ __global__ void __launch_bounds__(kMergeThreads) merge_kernel(const LayerArgs a,
   const int r = tid >> 3, c = tid & 7;  // piece row, 16-byte column of the 32-dim quarter
   const int nheads = a.B * a.Hkv;
   const int units = merge_units(nheads, a.G);
+  // The pieces of a head follow from the split of the concatenated token sets, which depends
+  // only on the head sizes: for layers of at most kMergeDirectHeads heads they are computed
+  // here, before the wait for the attention launch, from the lengths and the selection sizes.
+  // Both were complete before the attention launch passed its own wait, and this launch is
+  // only released by the attention launch after that point. Larger layers read the ranges the
+  // attention launch recorded, after the wait.
+  __shared__ long long mOff[kMergeDirectHeads + 1];
+  const bool direct = nheads <= kMergeDirectHeads;
+  if (direct && warp == 0) {
+    long long carry = 0;
+    for (int base = 0; base < nheads; base += 32) {
+      const int i = base + lane;
+      long long x = (i < nheads) ? head_len(a, w, i, nullptr) : 0;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const long long y = __shfl_up_sync(0xffffffffu, x, o);
+        if (lane >= o) x += y;
+      }
+      if (i < nheads) mOff[i + 1] = carry + x;
+      carry += __shfl_sync(0xffffffffu, x, 31);
+    }
+    if (lane == 0) mOff[0] = 0;
+  }
+  __syncthreads();
   pdl_wait();
   pdl_launch_dependents();
   for (int u = blockIdx.x; u < units; u += gridDim.x) {
     const int hd = u / (a.G * 4), jq = (u >> 2) % a.G, qtr = u & 3;
-    const int2 pr = __ldcg(w.head_pieces + hd);
-    const int c_first = pr.x, n = pr.y - pr.x + 1;
+    int c_first, n;
+    if (direct) {
+      const long long T = mOff[nheads];
+      const long long P = min((long long)a.attend_grid, T);
+      c_first = (int)cta_of(mOff[hd], T, P);
+      n = (int)cta_of(mOff[hd + 1] - 1, T, P) - c_first + 1;
+    } else {
+      const int2 pr = __ldcg(w.head_pieces + hd);
+      c_first = pr.x;
+      n = pr.y - pr.x + 1;
+    }
     if (n <= 1) continue;  // written by the attention launch
     const float* base = w.partials + (size_t)(c_first + hd) * kPartFloats;
     const int col = jq * kHeadDim + qtr * 32 + c * 4;

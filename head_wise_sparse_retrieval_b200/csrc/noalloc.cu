@@ -136,6 +136,7 @@ extern "C" rtp_status rtp_window_attention_noalloc(const rtp_noalloc_params* p, 
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   int grid = setup.num_sms * kAttendCtasPerSm;
   if (grid > kNaCtas) grid = kNaCtas;
+  a.attend_grid = grid;
   attend_kernel<<<grid, kAttendThreads, smem, s>>>(a, w);
   e = cudaGetLastError();
   if (e != cudaSuccess) return na_fail(RTP_ERR_CUDA, "attention kernel launch failed");

@@ -6,6 +6,8 @@
 #include <mutex>
 #include <vector>
 
+#include <nvtx3/nvToolsExt.h>
+
 #include "rtp.h"
 #include "rtp_device.cuh"
 #include "rtp_kernels.h"
@@ -49,6 +51,8 @@ struct rtp_handle {
   float step_p = 0.f;
   std::vector<const void*> step_ptrs;
   std::vector<uint8_t> step_masks;
+  // NVTX ranges around each call's launches (rtp_nvtx_enable)
+  bool nvtx = false;
   // kernel profiling (rtp_profile_enable)
   bool prof = false;
   std::vector<cudaEvent_t> prof_ev;   // 2 per launch
@@ -277,7 +281,8 @@ rtp_status enqueue_layer(rtp_handle* h, const LayerArgs& a0, cudaStream_t s, int
     if (e != cudaSuccess) return cuda_fail(e, "select_kernel launch");
   }
   if (withhold_cta >= 0) return RTP_OK;  // self-test: the selection alone
-  const LayerArgs& a = a0;
+  LayerArgs a = a0;
+  a.attend_grid = h->attend_grid;
   e = launch_one(h, 1, attend_kernel, dim3(h->attend_grid), dim3(kAttendThreads), h->attend_smem,
                  s, false, a, h->ws);
   if (e != cudaSuccess) return cuda_fail(e, "attend_kernel launch");
@@ -285,6 +290,21 @@ rtp_status enqueue_layer(rtp_handle* h, const LayerArgs& a0, cudaStream_t s, int
                  0, s, false, a, h->ws);
   return e == cudaSuccess ? RTP_OK : cuda_fail(e, "merge_kernel launch");
 }
+
+// An NVTX range around the launches of one call, when the handle has NVTX enabled (the ranges
+// cost nothing without a profiler attached, but stay off by default).
+struct NvtxRange {
+  bool on;
+  NvtxRange(const rtp_handle* h, const char* fmt, int x, int y) : on(h->nvtx) {
+    if (!on) return;
+    char name[96];
+    snprintf(name, sizeof name, fmt, x, y);
+    nvtxRangePushA(name);
+  }
+  ~NvtxRange() {
+    if (on) nvtxRangePop();
+  }
+};
 
 struct DeviceGuard {
   int prev = -1;
@@ -503,6 +523,7 @@ rtp_status rtp_decode_step(rtp_handle* h, int layer, const rtp_layer_io* io, voi
   rtp_status st = check_io(h, io, a.nret > 0);
   if (st != RTP_OK) return st;
   DeviceGuard guard(h->device);
+  NvtxRange range(h, "rtp_decode_step layer %d (%d retrieval KV heads)", layer, a.nret);
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   const bool single = io->single_launch != 0;
   st = single ? enqueue_fused(h, a, s, io->top_k) : enqueue_layer(h, a, s, io->top_k);
@@ -542,9 +563,10 @@ rtp_status rtp_indexer_append(rtp_handle* h, const rtp_indexer_io* io, void* str
     if (!io->head_mask || io->head_mask[k]) x.heads[x.nsel++] = (short)k;
   if (x.nsel == 0) return ok();
   DeviceGuard guard(h->device);
+  NvtxRange range(h, "rtp_indexer_append (%d x %d KV heads)", h->cfg.batch, x.nsel);
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(h->cfg.batch * x.nsel);
-  cfg.blockDim = dim3(128);
+  cfg.gridDim = dim3(h->cfg.batch * x.nsel * kIdxSplit);
+  cfg.blockDim = dim3(kIdxWarps * 32);
   cfg.stream = static_cast<cudaStream_t>(stream);
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
@@ -589,6 +611,7 @@ rtp_status rtp_dense_decode(rtp_handle* h, const rtp_layer_io* io, void* stream)
   a.dense = 1;
   a.nret = 0;
   DeviceGuard guard(h->device);
+  NvtxRange range(h, "rtp_dense_decode (%d x %d KV heads)", a.B, a.Hkv);
   st = enqueue_layer(h, a, static_cast<cudaStream_t>(stream));
   return st == RTP_OK ? ok() : st;
 }
@@ -773,6 +796,12 @@ rtp_status rtp_get_device_status(rtp_handle* h, uint32_t* code) {
   }
   if (e != cudaSuccess) return cuda_fail(e, "reading the device status");
   if (*code) return fail(RTP_ERR_DEVICE_STATUS, "device status 0x%x", *code);
+  return ok();
+}
+
+rtp_status rtp_nvtx_enable(rtp_handle* h, int enable) {
+  if (!h) return fail(RTP_ERR_INVALID_ARG, "handle is NULL");
+  h->nvtx = enable != 0;
   return ok();
 }
 

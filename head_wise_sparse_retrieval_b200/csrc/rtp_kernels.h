@@ -59,6 +59,7 @@ struct LayerArgs {
   float top_p, idx_scale, attn_scale_log2, bin_scale;
   short ret_kvh[kMaxKvHeads];     // KV head of retrieval index j (j < nret)
   short slot_of_kvh[kMaxKvHeads]; // retrieval index j of KV head kvh, or -1 for a local head
+  int attend_grid;                // CTAs of the attention launch (the merge derives the split)
   int early;                      // the caller vouches the inputs are complete before the
                                   // preceding launch ends: kernels may read them before waiting
 };
@@ -100,6 +101,8 @@ struct IndexerArgs {
   short heads[kMaxKvHeads];
 };
 __global__ void indexer_kernel(const IndexerArgs x);
+constexpr int kIdxWarps = 4;                             // outputs (one per warp) of a CTA
+constexpr int kIdxSplit = 16 / kIdxWarps;                // CTAs per (b, KV head): r = 16
 
 // Kernel entry points (defined in select_kernels.cu / attend_kernel.cu).
 // Cooperative launches. _onchip: every CTA's range fits in shared memory (no spill code);
@@ -128,6 +131,7 @@ constexpr int kHistCopies = 8;                           // copies of each slot'
 size_t select_smem_bytes(int slots);
 constexpr int kMaxPieces = 1024;                         // attention CTAs (pieces of one head)
 constexpr int kMergeThreads = 128;
+constexpr int kMergeDirectHeads = 64;                    // heads whose pieces the merge derives
 // merge units: (head, query head of the group, quarter of the 128 dimensions)
 __host__ __device__ inline int merge_units(int nheads, int G) { return nheads * G * 4; }
 

@@ -25,7 +25,7 @@ EXPORTS = ("rtp_config_default", "rtp_workspace_bytes", "rtp_create", "rtp_destr
            "rtp_decode_step", "rtp_dense_decode", "rtp_decode_step_host", "rtp_get_selection",
            "rtp_get_threshold", "rtp_get_device_status", "rtp_status_string", "rtp_last_error",
            "rtp_profile_enable", "rtp_profile_read", "rtp_window_attention_noalloc",
-           "rtp_indexer_append", "rtp_selftest_wait_timeout")
+           "rtp_indexer_append", "rtp_selftest_wait_timeout", "rtp_nvtx_enable")
 NOALLOC_MAX_HEADS = 64
 KERNEL_CLASSES = ("select", "attend", "merge", "fused")
 
@@ -102,6 +102,7 @@ def load(path: str = LIB_PATH):
                                     ctypes.POINTER(ctypes.c_float)]
     L.rtp_get_device_status.argtypes = [vp, ctypes.POINTER(ctypes.c_uint32)]
     L.rtp_profile_enable.argtypes = [vp, i]
+    L.rtp_nvtx_enable.argtypes = [vp, i]
     L.rtp_profile_read.argtypes = [vp, ctypes.POINTER(ctypes.c_double),
                                    ctypes.POINTER(ctypes.c_int64)]
     L.rtp_window_attention_noalloc.argtypes = [ctypes.POINTER(NoAllocParams), vp, vp, vp, vp,
@@ -274,6 +275,10 @@ class Handle:
 
     def profile(self, enable: bool):
         _check(load().rtp_profile_enable(self._h, int(bool(enable))), "rtp_profile_enable")
+
+    def nvtx(self, enable: bool):
+        """rtp_nvtx_enable: one NVTX range per call around its launches (off by default)."""
+        _check(load().rtp_nvtx_enable(self._h, int(bool(enable))), "rtp_nvtx_enable")
 
     def profile_read(self) -> dict:
         """{class: (total ms, launches)} for the launches recorded since the last read."""

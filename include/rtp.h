@@ -161,8 +161,11 @@ RTP_API rtp_status rtp_decode_step(rtp_handle *h, int layer, const rtp_layer_io 
  *   k_idx[b][h][N_b-1][i]  = fp16( sum_{d < D}   w_k[h][i][d] * k_pre[b][h][d] )
  * (the G query heads of the KV head's group concatenated head-major; fp32 accumulation,
  * rounded to nearest fp16 once). All pointers are device memory, 16-byte aligned except
- * seq_lens (4). Errors: RTP_ERR_INVALID_ARG for NULL / misaligned pointers; a seq_lens entry
- * outside [1, max_ctx] is clamped and reported in the device status word. */
+ * seq_lens (4). The weights w_q and w_k are read before the kernel waits for the preceding
+ * launch on the stream, so that launch must not write them (model weights are constant
+ * during decode); q_pre, k_pre and seq_lens are read after the wait. Errors:
+ * RTP_ERR_INVALID_ARG for NULL / misaligned pointers; a seq_lens entry outside [1, max_ctx]
+ * is clamped and reported in the device status word. */
 typedef struct {
     const void *q_pre;       /* bf16 [B][Hq][D]: pre-RoPE queries of the current token         */
     const void *k_pre;       /* bf16 [B][Hkv][D]: pre-RoPE key of the current token            */
@@ -217,6 +220,14 @@ RTP_API rtp_status rtp_get_threshold(rtp_handle *h, int b, int kvh, int *bstar, 
  * (rtp_layer_io.single_launch). The event pool holds 1024
  * launches; rtp_profile_read empties it. Errors: RTP_ERR_CUDA if the events cannot be created. */
 RTP_API rtp_status rtp_profile_enable(rtp_handle *h, int enable);
+
+/* NVTX ranges. While enabled (off by default), every rtp_decode_step, rtp_dense_decode and
+ * rtp_indexer_append call on this handle pushes one NVTX range around its launches, named for
+ * the call, the layer and its retrieval-head count ("rtp_decode_step layer 7 (1 retrieval KV
+ * heads)"), so that a timeline profiler shows each layer's kernels under one label. The
+ * ranges are host-side markers: they cost nothing without a profiler attached and are legal
+ * during stream capture. Errors: RTP_ERR_INVALID_ARG for a NULL handle. */
+RTP_API rtp_status rtp_nvtx_enable(rtp_handle *h, int enable);
 
 /* Synchronises the recorded launches, adds their durations (ms) and counts per kernel class
  * into ms[4] and launches[4] (overwritten), and empties the pool. */
