@@ -844,6 +844,28 @@ rtp_status rtp_profile_read(rtp_handle* h, double* ms, int64_t* launches) {
   return ok();
 }
 
+rtp_status rtp_profile_launches(rtp_handle* h, double* ms, int32_t* kind, int64_t cap,
+                                int64_t* count) {
+  if (!h || !count || (cap > 0 && (!ms || !kind)))
+    return fail(RTP_ERR_INVALID_ARG, "NULL argument");
+  DeviceGuard guard(h->device);
+  const int n = h->prof_used;
+  *count = n;
+  for (int i = 0; i < n && i < cap; ++i) {
+    float t = 0.f;
+    cudaError_t e = cudaEventSynchronize(h->prof_ev[2 * i + 1]);
+    if (e == cudaSuccess) e = cudaEventElapsedTime(&t, h->prof_ev[2 * i], h->prof_ev[2 * i + 1]);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaEventElapsedTime");
+    ms[i] = t;
+    kind[i] = h->prof_kind[i];
+  }
+  const bool overflow = h->prof_overflow || n > cap;
+  h->prof_used = 0;
+  h->prof_overflow = false;
+  if (overflow) return fail(RTP_ERR_INVALID_ARG, "more launches recorded than cap (or the pool)");
+  return ok();
+}
+
 const char* rtp_status_string(rtp_status s) {
   switch (s) {
     case RTP_OK: return "RTP_OK";

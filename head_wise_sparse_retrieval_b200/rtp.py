@@ -25,7 +25,8 @@ EXPORTS = ("rtp_config_default", "rtp_workspace_bytes", "rtp_create", "rtp_destr
            "rtp_decode_step", "rtp_dense_decode", "rtp_decode_step_host", "rtp_get_selection",
            "rtp_get_threshold", "rtp_get_device_status", "rtp_status_string", "rtp_last_error",
            "rtp_profile_enable", "rtp_profile_read", "rtp_window_attention_noalloc",
-           "rtp_indexer_append", "rtp_selftest_wait_timeout", "rtp_nvtx_enable")
+           "rtp_indexer_append", "rtp_selftest_wait_timeout", "rtp_nvtx_enable",
+           "rtp_profile_launches")
 NOALLOC_MAX_HEADS = 64
 KERNEL_CLASSES = ("select", "attend", "merge", "fused")
 
@@ -105,6 +106,9 @@ def load(path: str = LIB_PATH):
     L.rtp_nvtx_enable.argtypes = [vp, i]
     L.rtp_profile_read.argtypes = [vp, ctypes.POINTER(ctypes.c_double),
                                    ctypes.POINTER(ctypes.c_int64)]
+    L.rtp_profile_launches.argtypes = [vp, ctypes.POINTER(ctypes.c_double),
+                                       ctypes.POINTER(ctypes.c_int32), ctypes.c_int64,
+                                       ctypes.POINTER(ctypes.c_int64)]
     L.rtp_window_attention_noalloc.argtypes = [ctypes.POINTER(NoAllocParams), vp, vp, vp, vp,
                                                vp, vp]
     L.rtp_window_attention_noalloc.restype = ctypes.c_int
@@ -286,6 +290,15 @@ class Handle:
         n = (ctypes.c_int64 * 4)()
         _check(load().rtp_profile_read(self._h, ms, n), "rtp_profile_read")
         return {k: (ms[i], int(n[i])) for i, k in enumerate(KERNEL_CLASSES)}
+
+    def profile_launches(self, cap: int = 1024) -> list:
+        """[(class, ms)] of the launches recorded since the last read, in launch order."""
+        ms = (ctypes.c_double * cap)()
+        kind = (ctypes.c_int32 * cap)()
+        n = ctypes.c_int64()
+        _check(load().rtp_profile_launches(self._h, ms, kind, cap, ctypes.byref(n)),
+               "rtp_profile_launches")
+        return [(KERNEL_CLASSES[kind[i]], ms[i]) for i in range(n.value)]
 
     def device_status(self) -> int:
         code = ctypes.c_uint32()

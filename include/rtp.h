@@ -221,6 +221,13 @@ RTP_API rtp_status rtp_get_threshold(rtp_handle *h, int b, int kvh, int *bstar, 
  * launches; rtp_profile_read empties it. Errors: RTP_ERR_CUDA if the events cannot be created. */
 RTP_API rtp_status rtp_profile_enable(rtp_handle *h, int enable);
 
+/* The same recorded launches one by one, in launch order: ms[i] and kind[i] (the classes of
+ * rtp_profile_read) for i < min(cap, *count), *count = the number recorded. Synchronises them
+ * and empties the pool. Errors: RTP_ERR_INVALID_ARG for NULL arguments, or when more launches
+ * were recorded than cap (the first cap are still written) or than the pool holds. */
+RTP_API rtp_status rtp_profile_launches(rtp_handle *h, double *ms, int32_t *kind, int64_t cap,
+                                        int64_t *count);
+
 /* NVTX ranges. While enabled (off by default), every rtp_decode_step, rtp_dense_decode and
  * rtp_indexer_append call on this handle pushes one NVTX range around its launches, named for
  * the call, the layer and its retrieval-head count ("rtp_decode_step layer 7 (1 retrieval KV

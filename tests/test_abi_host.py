@@ -88,6 +88,9 @@ def test_calls_on_null_handle_are_rejected(rtp_lib):
     assert L.rtp_selftest_wait_timeout(None, 0, ctypes.byref(io), 1000000, None) == \
         rtp_lib.RTP_ERR_INVALID_ARG
     assert L.rtp_nvtx_enable(None, 1) == rtp_lib.RTP_ERR_INVALID_ARG
+    n = ctypes.c_int64()
+    assert L.rtp_profile_launches(None, None, None, 0, ctypes.byref(n)) == \
+        rtp_lib.RTP_ERR_INVALID_ARG
     assert L.rtp_destroy(None) == rtp_lib.RTP_OK
     assert L.rtp_status_string(3) == b"RTP_ERR_OOM"
 

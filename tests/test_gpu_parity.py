@@ -413,3 +413,27 @@ def test_maximum_head_count():
                  retrieval=ret, kinds=kinds, n_needles=needles, seed=17)
     heads = [(b, k) for b in (0, 1, 31, 62, 63) for k in (0, 3, 4, 12, 15)]
     _run(p, heads=heads, exact=False)
+
+
+def test_profiling_and_nvtx_do_not_change_results():
+    """Per-launch events (rtp_profile_launches) report each layer's launches in order, and
+    neither they nor NVTX ranges change the outputs (bit-equal to a plain run)."""
+    p = W.custom(batch=2, num_q_heads=32, num_kv_heads=4, seq_lens=[20000, 9000],
+                 max_ctx=20000, retrieval=[1, 0, 1, 0],
+                 kinds=[[W.KIND_DIFFUSE, 0, W.KIND_CONC, 0]] * 2, n_needles=[[0, 0, 4, 0]] * 2,
+                 seed=23)
+    li = W.make_layer(p, 0, DEV)
+    with make_handle(p) as h:
+        plain, _ = run_layer(h, p, li, 0)
+        h.profile(True)
+        h.nvtx(True)
+        profiled, _ = run_layer(h, p, li, 0)
+        dense, _ = run_layer(h, p, li, 0, dense=True)
+        launches = h.profile_launches()
+        h.profile(False)
+        h.nvtx(False)
+    assert torch.equal(plain, profiled)
+    assert [k for k, _ in launches] == ["select", "attend", "merge", "attend", "merge"]
+    assert all(ms > 0 for _, ms in launches)
+    check_output(dense.cpu().numpy()[0, 0:8], oracle_head(li, 0, 0, False, 0.9, 8,
+                                                          dense=True).out, "dense after profiling")
