@@ -21,6 +21,7 @@
 // At the end of a head's piece the warps merge (m, l, O) through shared memory. A head held by
 // one CTA is written out there; a head split over several CTAs leaves one partial per CTA, and
 // merge_kernel (the next launch on the stream) combines them by log-sum-exp in a fixed order.
+#include "attend_tile.cuh"
 #include "rtp_device.cuh"
 #include "rtp_kernels.h"
 
@@ -29,9 +30,7 @@ namespace rtp {
 namespace {
 
 constexpr int kWarps = kAttendWarps;
-constexpr int kTile = 16;
 constexpr int kDepth = kAttendDepth;
-constexpr int kWarpStage = 2 * kTile * kRowBytes;          // 16 K rows then 16 V rows
 constexpr int kOPitch = kHeadDim + 4;                      // padded row of the merge buffer
 constexpr int kCombFloats = kMaxGroup * kOPitch + kWarps * kMaxGroup * 2 + kMaxGroup * 2;
 constexpr int kMergeRows = kMergeThreads / 8;              // pieces a merge pass loads at once
@@ -48,19 +47,6 @@ struct SmemLayout {
     return seq_off(nheads) + (size_t)batch * 4;
   }
 };
-
-// Byte offset of 16-byte column c of row r inside a stage: rows are 256 B, the column is
-// XOR-swizzled with the row so that the 8 rows an ldmatrix reads hit 8 different bank groups.
-__device__ __forceinline__ uint32_t swz(int r, int c) {
-  return (uint32_t)(r * kRowBytes + ((c ^ (r & 7)) << 4));
-}
-
-__device__ __forceinline__ int window_len(int N, int W, int S) {
-  return (N <= W + S) ? N : W + S;
-}
-__device__ __forceinline__ int window_pos(int r, int N, int W, int S) {
-  return (N <= W + S) ? r : (r < S ? r : N - W + (r - S));
-}
 
 // Size of head hd's token set (retrieval: |S| from the selection, clamped to [1, N]; local:
 // the window set; dense: N), N = seq_lens[b] clamped to [1, max_ctx]. The attention split and
@@ -170,33 +156,11 @@ __device__ __forceinline__ int tile_positions(const HeadRef& h, const LayerArgs&
   return h.window ? window_pos(rank, h.N, a.window, a.sinks) : rank;
 }
 
-// Gathers the tile's K and V rows into the stage: lane l copies 16-byte column c = l % 16 of
-// rows 2i + l / 16; the positions come from lanes 0..15 of pos. A position outside [0, N) (a
-// corrupted list) is replaced by 0 and reported once per tile; rows past n are zero-filled.
+// Gathers the tile's K and V rows into the stage (attend_tile.cuh): rows past n are
+// zero-filled, a position outside [0, N) is replaced by 0 and reported.
 __device__ __forceinline__ void issue_tile(uint32_t stage, const HeadRef& h, int pos, int n,
                                            int lane, uint64_t policy, unsigned* status) {
-  const int c = lane & 15, par = lane >> 4;
-  // swz(2i + par, c) = (2i + par) * 256 + ((c ^ ((2i + par) & 7)) << 4)
-  //                  = par * 256 + 512 i + (((c ^ par) ^ 2 (i & 3)) << 4)
-  const uint32_t lane_base = stage + (uint32_t)par * kRowBytes;
-  const int cx = c ^ par;
-  const __nv_bfloat16* kcol = h.kbase + c * 8;
-  const __nv_bfloat16* vcol = h.vbase + c * 8;
-  bool bad = false;
-#pragma unroll
-  for (int i = 0; i < kTile / 2; ++i) {
-    const int row = 2 * i + par;
-    const int p = __shfl_sync(0xffffffffu, pos, row);
-    const bool valid = row < n;
-    const bool in = (unsigned)p < (unsigned)h.N;
-    bad |= valid && !in;
-    const size_t off = (valid && in) ? (size_t)p * kHeadDim : 0;
-    const unsigned bytes = valid ? 16u : 0u;
-    const uint32_t dst = lane_base + 512u * i + ((uint32_t)(cx ^ (2 * (i & 3))) << 4);
-    cp_async_16(dst, kcol + off, bytes, policy);
-    cp_async_16(dst + kTile * kRowBytes, vcol + off, bytes, policy);
-  }
-  if (__any_sync(0xffffffffu, bad) && lane == 0) atomicOr(status, kDevBadIndex);
+  gather_tile(stage, h.kbase, h.vbase, h.N, pos, n, lane, policy, status);
 }
 
 }  // namespace
@@ -315,9 +279,6 @@ __global__ void __launch_bounds__(kAttendThreads, kAttendCtasPerSm) attend_kerne
   // ---- math side: segment by segment ----
   const int g = lane >> 2, t = lane & 3;  // MMA fragment coordinates
   const float scale_log2 = a.attn_scale_log2;
-  // ldmatrix rows / 16-byte columns this lane addresses (before the swizzle)
-  const int k_row = (lane & 7) + ((lane >> 3) & 1) * 8, k_col = lane >> 4;
-  const int v_row = kTile + (lane & 7) + (lane >> 4) * 8, v_col = (lane >> 3) & 1;
   int done = 0;     // warp tiles computed
   int kseg = 0;     // global tile index of the current segment's first tile
   Walk walk;
@@ -326,22 +287,10 @@ __global__ void __launch_bounds__(kAttendThreads, kAttendCtasPerSm) attend_kerne
   while (walk.next(hd, r0, r1)) {
     const int nt = (r1 - r0 + kTile - 1) / kTile;
     const int b = hd / a.Hkv, kvh = hd - b * a.Hkv;
-    // Q^T as the B operand: b0 = q[g][16ks + 2t, +1], b1 = q[g][16ks + 8 + 2t, +1]
     uint32_t qf[8][2];
-    {
-      const bool valid = g < a.G;
-      const uint32_t* qrow = reinterpret_cast<const uint32_t*>(
-          a.q + ((size_t)b * a.Hq + (size_t)kvh * a.G + (valid ? g : 0)) * kHeadDim);
-#pragma unroll
-      for (int ks = 0; ks < 8; ++ks) {
-        qf[ks][0] = valid ? qrow[ks * 8 + t] : 0u;
-        qf[ks][1] = valid ? qrow[ks * 8 + 4 + t] : 0u;
-      }
-    }
-    float m0 = -INFINITY, m1 = -INFINITY, l0 = 0.f, l1 = 0.f;
-    float acc[8][4];
-#pragma unroll
-    for (int mt = 0; mt < 8; ++mt) acc[mt][0] = acc[mt][1] = acc[mt][2] = acc[mt][3] = 0.f;
+    load_q_frag(qf, a.q + ((size_t)b * a.Hq + (size_t)kvh * a.G) * kHeadDim, a.G, lane);
+    TileAcc st;
+    st.init();
 
     for (int k = warp + kWarps * done; k < kseg + nt; k += kWarps, ++done) {
       // keep kDepth - 1 tiles in flight: issue warp tile done + kDepth - 1, then prefetch the
@@ -353,57 +302,7 @@ __global__ void __launch_bounds__(kAttendThreads, kAttendCtasPerSm) attend_kerne
       __syncwarp();
 
       const int n = min(kTile, r1 - (r0 + (k - kseg) * kTile));  // valid tokens of this tile
-      const uint32_t kb = my_stages + (done % kDepth) * kWarpStage;
-      // S^T (16 tokens x 8 heads) = K (16 x 128) . Q^T (128 x 8), two accumulator chains
-      float sa[4] = {0.f, 0.f, 0.f, 0.f}, sb[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-      for (int ks = 0; ks < 8; ks += 2) {
-        uint32_t fa[4], fb[4];
-        ldmatrix_x4(fa, kb + swz(k_row, 2 * ks + k_col));
-        ldmatrix_x4(fb, kb + swz(k_row, 2 * ks + 2 + k_col));
-        mma_bf16_16816(sa, fa, qf[ks][0], qf[ks][1]);
-        mma_bf16_16816(sb, fb, qf[ks + 1][0], qf[ks + 1][1]);
-      }
-      // rows: token g (c0: head 2t, c1: head 2t+1) and token g+8 (c2, c3)
-      float x0 = (sa[0] + sb[0]) * scale_log2, x1 = (sa[1] + sb[1]) * scale_log2;
-      float x2 = (sa[2] + sb[2]) * scale_log2, x3 = (sa[3] + sb[3]) * scale_log2;
-      if (g >= n) x0 = x1 = -INFINITY;
-      if (g + 8 >= n) x2 = x3 = -INFINITY;
-      float mx0 = fmaxf(x0, x2), mx1 = fmaxf(x1, x3);
-#pragma unroll
-      for (int o = 4; o < 32; o <<= 1) {
-        mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, o));
-        mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, o));
-      }
-      const float mn0 = fmaxf(m0, mx0), mn1 = fmaxf(m1, mx1);  // finite: token 0 is valid
-      if (__any_sync(0xffffffffu, mn0 > m0 || mn1 > m1)) {  // rescale only when a max grows
-        const float al0 = exp2f(m0 - mn0), al1 = exp2f(m1 - mn1);
-        l0 *= al0;
-        l1 *= al1;
-#pragma unroll
-        for (int mt = 0; mt < 8; ++mt) {
-          acc[mt][0] *= al0;
-          acc[mt][1] *= al1;
-          acc[mt][2] *= al0;
-          acc[mt][3] *= al1;
-        }
-        m0 = mn0;
-        m1 = mn1;
-      }
-      const uint32_t p01 = pack_bf16x2(exp2f(x0 - m0), exp2f(x1 - m1));
-      const uint32_t p23 = pack_bf16x2(exp2f(x2 - m0), exp2f(x3 - m1));
-      l0 += bf16_lo(p01) + bf16_lo(p23);
-      l1 += bf16_hi(p01) + bf16_hi(p23);
-      // P^T as the B operand: transpose the 8x8 (token x head) blocks in registers
-      const uint32_t pb0 = movmatrix_trans(p01);
-      const uint32_t pb1 = movmatrix_trans(p23);
-      // O^T (128 dims x 8 heads) += V^T (128 x 16 tokens) . P^T (16 x 8)
-#pragma unroll
-      for (int mt = 0; mt < 8; ++mt) {
-        uint32_t fv[4];
-        ldmatrix_x4_trans(fv, kb + swz(v_row, 2 * mt + v_col));
-        mma_bf16_16816(acc[mt], fv, pb0, pb1);
-      }
+      attend_tile(my_stages + (done % kDepth) * kWarpStage, qf, n, scale_log2, lane, st);
       __syncwarp();  // the stage is refilled kDepth - 1 tiles later
     }
     kseg += nt;
@@ -416,14 +315,14 @@ __global__ void __launch_bounds__(kAttendThreads, kAttendCtasPerSm) attend_kerne
     float* sML = sComb + kMaxGroup * kOPitch;            // [kWarps][8][2]
 #pragma unroll
     for (int o = 4; o < 32; o <<= 1) {
-      l0 += __shfl_xor_sync(0xffffffffu, l0, o);
-      l1 += __shfl_xor_sync(0xffffffffu, l1, o);
+      st.l0 += __shfl_xor_sync(0xffffffffu, st.l0, o);
+      st.l1 += __shfl_xor_sync(0xffffffffu, st.l1, o);
     }
     if (g == 0) {
-      sML[(warp * kMaxGroup + 2 * t) * 2] = m0;
-      sML[(warp * kMaxGroup + 2 * t) * 2 + 1] = l0;
-      sML[(warp * kMaxGroup + 2 * t + 1) * 2] = m1;
-      sML[(warp * kMaxGroup + 2 * t + 1) * 2 + 1] = l1;
+      sML[(warp * kMaxGroup + 2 * t) * 2] = st.m0;
+      sML[(warp * kMaxGroup + 2 * t) * 2 + 1] = st.l0;
+      sML[(warp * kMaxGroup + 2 * t + 1) * 2] = st.m1;
+      sML[(warp * kMaxGroup + 2 * t + 1) * 2 + 1] = st.l1;
     }
     __syncthreads();
     {
@@ -433,8 +332,8 @@ __global__ void __launch_bounds__(kAttendThreads, kAttendCtasPerSm) attend_kerne
         M0 = fmaxf(M0, sML[(wq * kMaxGroup + 2 * t) * 2]);
         M1 = fmaxf(M1, sML[(wq * kMaxGroup + 2 * t + 1) * 2]);
       }
-      const float f0 = (m0 == -INFINITY) ? 0.f : exp2f(m0 - M0);  // 0: a warp without tokens
-      const float f1 = (m1 == -INFINITY) ? 0.f : exp2f(m1 - M1);
+      const float f0 = (st.m0 == -INFINITY) ? 0.f : exp2f(st.m0 - M0);  // 0: a warp without tokens
+      const float f1 = (st.m1 == -INFINITY) ? 0.f : exp2f(st.m1 - M1);
 #pragma unroll
       for (int wq = 0; wq < kWarps; ++wq) {
         if (warp == wq) {
@@ -443,15 +342,15 @@ __global__ void __launch_bounds__(kAttendThreads, kAttendCtasPerSm) attend_kerne
             float* r0p = sO + (2 * t) * kOPitch + 16 * mt + g;
             float* r1p = sO + (2 * t + 1) * kOPitch + 16 * mt + g;
             if (wq == 0) {
-              r0p[0] = acc[mt][0] * f0;
-              r1p[0] = acc[mt][1] * f1;
-              r0p[8] = acc[mt][2] * f0;
-              r1p[8] = acc[mt][3] * f1;
+              r0p[0] = st.acc[mt][0] * f0;
+              r1p[0] = st.acc[mt][1] * f1;
+              r0p[8] = st.acc[mt][2] * f0;
+              r1p[8] = st.acc[mt][3] * f1;
             } else {
-              r0p[0] += acc[mt][0] * f0;
-              r1p[0] += acc[mt][1] * f1;
-              r0p[8] += acc[mt][2] * f0;
-              r1p[8] += acc[mt][3] * f1;
+              r0p[0] += st.acc[mt][0] * f0;
+              r1p[0] += st.acc[mt][1] * f1;
+              r0p[8] += st.acc[mt][2] * f0;
+              r1p[8] += st.acc[mt][3] * f1;
             }
           }
         }

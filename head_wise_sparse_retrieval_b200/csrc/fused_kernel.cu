@@ -33,6 +33,7 @@
 //   phase 5    (grid barrier) the CTAs merge the split heads by log-sum-exp, one (head, query
 //              head, 32 dimensions) unit at a time, every sum in a fixed order.
 // All waits are bounded (kDevWaitTimeout); after a timed-out barrier the CTA stops.
+#include "attend_tile.cuh"
 #include "rtp_device.cuh"
 #include "rtp_kernels.h"
 
@@ -42,11 +43,9 @@ namespace {
 
 constexpr int kW = kFusedWarps;
 constexpr int kT = kFusedThreads;
-constexpr int kTile = 16;                                  // tokens per MMA tile
 constexpr int kDepth = 3;                                  // gather stages per warp
 constexpr int kOwn = kFusedOwnTok;
 constexpr int kRing = 4;                                   // indexer-key stages per warp
-constexpr int kWarpStage = 2 * kTile * kRowBytes;          // 16 K rows, then 16 V rows
 constexpr int kRegion = kW * kDepth * kWarpStage;          // 192 KB, reused by every phase
 constexpr int kKeyStage = kOwn * kIdxDim * 2;              // one tile of indexer keys (2 KB)
 constexpr int kRingBytes = kW * kRing * kKeyStage;         // phase 1: [0, 64 KB)
@@ -71,13 +70,6 @@ static_assert(kFusedCapTiles <= 2 * kT, "the popcount prefix takes two tiles per
 static_assert(kT == kBins, "phase 2 flushes one bin per thread");
 static_assert(2 * 1024 * 4 + 256 + kW * 8 * 16 <= kRegion, "merge arrays fit the region");
 
-__device__ __forceinline__ uint32_t swz(int r, int c) {
-  return (uint32_t)(r * kRowBytes + ((c ^ (r & 7)) << 4));
-}
-__device__ __forceinline__ int window_len(int N, int W, int S) { return (N <= W + S) ? N : W + S; }
-__device__ __forceinline__ int window_pos(int r, int N, int W, int S) {
-  return (N <= W + S) ? r : (r < S ? r : N - W + (r - S));
-}
 
 // Position of the k-th (0-based) set bit of x, k < popc(x): halving the window by popcounts.
 __device__ __forceinline__ int nth_set32(unsigned x, int k) {
@@ -148,31 +140,10 @@ struct HeadRef {
   int N;
 };
 
-// Gathers the tile's K and V rows into the stage (rows past n are zero-filled): lane l copies
-// 16-byte column l % 16 of rows 2i + l / 16, positions from lanes 0..15 of pos. A position
-// outside [0, N) is replaced by 0 and reported.
+// Gathers the tile's K and V rows into the stage (attend_tile.cuh).
 __device__ __forceinline__ void issue_tile(uint32_t stage, const HeadRef& h, int pos, int n,
                                            int lane, uint64_t policy, unsigned* status) {
-  const int c = lane & 15, par = lane >> 4;
-  const uint32_t lane_base = stage + (uint32_t)par * kRowBytes;
-  const int cx = c ^ par;
-  const __nv_bfloat16* kcol = h.kbase + c * 8;
-  const __nv_bfloat16* vcol = h.vbase + c * 8;
-  bool bad = false;
-#pragma unroll
-  for (int i = 0; i < kTile / 2; ++i) {
-    const int row = 2 * i + par;
-    const int p = __shfl_sync(0xffffffffu, pos, row);
-    const bool valid = row < n;
-    const bool in = (unsigned)p < (unsigned)h.N;
-    bad |= valid && !in;
-    const size_t off = (valid && in) ? (size_t)p * kHeadDim : 0;
-    const unsigned bytes = valid ? 16u : 0u;
-    const uint32_t dst = lane_base + 512u * i + ((uint32_t)(cx ^ (2 * (i & 3))) << 4);
-    cp_async_16(dst, kcol + off, bytes, policy);
-    cp_async_16(dst + kTile * kRowBytes, vcol + off, bytes, policy);
-  }
-  if (__any_sync(0xffffffffu, bad) && lane == 0) atomicOr(status, kDevBadIndex);
+  gather_tile(stage, h.kbase, h.vbase, h.N, pos, n, lane, policy, status);
 }
 
 // Per-CTA tables, built in the prologue.
@@ -696,8 +667,6 @@ __global__ void __launch_bounds__(kT, 1) fused_layer_kernel(const LayerArgs a, c
   // math side: the same units in the same order
   const int g = lane >> 2, t = lane & 3;  // MMA fragment coordinates
   const float scale_log2 = a.attn_scale_log2;
-  const int k_row = (lane & 7) + ((lane >> 3) & 1) * 8, k_col = lane >> 4;
-  const int v_row = kTile + (lane & 7) + (lane >> 4) * 8, v_col = (lane >> 3) & 1;
   int done = 0;
   UnitWalk mw;
   mw.begin(tb, lt0, lt1);
@@ -705,73 +674,16 @@ __global__ void __launch_bounds__(kT, 1) fused_layer_kernel(const LayerArgs a, c
   while (mw.next(tb, a, pre, S, warp, u)) {
     const int b = u.hd / a.Hkv, kvh = u.hd - b * a.Hkv;
     uint32_t qf[8][2];
-    {
-      const bool valid = g < a.G;
-      const uint32_t* qrow = reinterpret_cast<const uint32_t*>(
-          a.q + ((size_t)b * a.Hq + (size_t)kvh * a.G + (valid ? g : 0)) * kHeadDim);
-#pragma unroll
-      for (int ks = 0; ks < 8; ++ks) {
-        qf[ks][0] = valid ? qrow[ks * 8 + t] : 0u;
-        qf[ks][1] = valid ? qrow[ks * 8 + 4 + t] : 0u;
-      }
-    }
-    float m0 = -INFINITY, m1 = -INFINITY, l0 = 0.f, l1 = 0.f;
-    float acc[8][4];
-#pragma unroll
-    for (int mt = 0; mt < 8; ++mt) acc[mt][0] = acc[mt][1] = acc[mt][2] = acc[mt][3] = 0.f;
+    load_q_frag(qf, a.q + ((size_t)b * a.Hq + (size_t)kvh * a.G) * kHeadDim, a.G, lane);
+    TileAcc st;
+    st.init();
     const int len_w = u.rb - u.ra;
     for (int r = 0; r < len_w; r += kTile, ++done) {
       issue(done + kDepth - 1);
       cp_async_wait<kDepth - 1>();
       __syncwarp();
       const int n = min(kTile, len_w - r);
-      const uint32_t kb = my_stages + (done % kDepth) * kWarpStage;
-      float sa[4] = {0.f, 0.f, 0.f, 0.f}, sb[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-      for (int ks = 0; ks < 8; ks += 2) {
-        uint32_t fa[4], fb[4];
-        ldmatrix_x4(fa, kb + swz(k_row, 2 * ks + k_col));
-        ldmatrix_x4(fb, kb + swz(k_row, 2 * ks + 2 + k_col));
-        mma_bf16_16816(sa, fa, qf[ks][0], qf[ks][1]);
-        mma_bf16_16816(sb, fb, qf[ks + 1][0], qf[ks + 1][1]);
-      }
-      float x0 = (sa[0] + sb[0]) * scale_log2, x1 = (sa[1] + sb[1]) * scale_log2;
-      float x2 = (sa[2] + sb[2]) * scale_log2, x3 = (sa[3] + sb[3]) * scale_log2;
-      if (g >= n) x0 = x1 = -INFINITY;
-      if (g + 8 >= n) x2 = x3 = -INFINITY;
-      float mx0 = fmaxf(x0, x2), mx1 = fmaxf(x1, x3);
-#pragma unroll
-      for (int o = 4; o < 32; o <<= 1) {
-        mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, o));
-        mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, o));
-      }
-      const float mn0 = fmaxf(m0, mx0), mn1 = fmaxf(m1, mx1);  // finite: token 0 is valid
-      if (__any_sync(0xffffffffu, mn0 > m0 || mn1 > m1)) {
-        const float al0 = exp2f(m0 - mn0), al1 = exp2f(m1 - mn1);
-        l0 *= al0;
-        l1 *= al1;
-#pragma unroll
-        for (int mt = 0; mt < 8; ++mt) {
-          acc[mt][0] *= al0;
-          acc[mt][1] *= al1;
-          acc[mt][2] *= al0;
-          acc[mt][3] *= al1;
-        }
-        m0 = mn0;
-        m1 = mn1;
-      }
-      const uint32_t p01 = pack_bf16x2(exp2f(x0 - m0), exp2f(x1 - m1));
-      const uint32_t p23 = pack_bf16x2(exp2f(x2 - m0), exp2f(x3 - m1));
-      l0 += bf16_lo(p01) + bf16_lo(p23);
-      l1 += bf16_hi(p01) + bf16_hi(p23);
-      const uint32_t pb0 = movmatrix_trans(p01);
-      const uint32_t pb1 = movmatrix_trans(p23);
-#pragma unroll
-      for (int mt = 0; mt < 8; ++mt) {
-        uint32_t fv[4];
-        ldmatrix_x4_trans(fv, kb + swz(v_row, 2 * mt + v_col));
-        mma_bf16_16816(acc[mt], fv, pb0, pb1);
-      }
+      attend_tile(my_stages + (done % kDepth) * kWarpStage, qf, n, scale_log2, lane, st);
       __syncwarp();  // the stage is refilled kDepth - 1 tiles later
     }
 
@@ -790,14 +702,14 @@ __global__ void __launch_bounds__(kT, 1) fused_layer_kernel(const LayerArgs a, c
     float* sML = sComb + kMaxGroup * kOPitch;            // [kW][8][2]
 #pragma unroll
     for (int o = 4; o < 32; o <<= 1) {
-      l0 += __shfl_xor_sync(0xffffffffu, l0, o);
-      l1 += __shfl_xor_sync(0xffffffffu, l1, o);
+      st.l0 += __shfl_xor_sync(0xffffffffu, st.l0, o);
+      st.l1 += __shfl_xor_sync(0xffffffffu, st.l1, o);
     }
     if (g == 0) {
-      sML[(warp * kMaxGroup + 2 * t) * 2] = m0;
-      sML[(warp * kMaxGroup + 2 * t) * 2 + 1] = l0;
-      sML[(warp * kMaxGroup + 2 * t + 1) * 2] = m1;
-      sML[(warp * kMaxGroup + 2 * t + 1) * 2 + 1] = l1;
+      sML[(warp * kMaxGroup + 2 * t) * 2] = st.m0;
+      sML[(warp * kMaxGroup + 2 * t) * 2 + 1] = st.l0;
+      sML[(warp * kMaxGroup + 2 * t + 1) * 2] = st.m1;
+      sML[(warp * kMaxGroup + 2 * t + 1) * 2 + 1] = st.l1;
     }
     __syncthreads();
     {
@@ -807,8 +719,8 @@ __global__ void __launch_bounds__(kT, 1) fused_layer_kernel(const LayerArgs a, c
         M0 = fmaxf(M0, sML[(wq * kMaxGroup + 2 * t) * 2]);
         M1 = fmaxf(M1, sML[(wq * kMaxGroup + 2 * t + 1) * 2]);
       }
-      const float f0 = (m0 == -INFINITY) ? 0.f : exp2f(m0 - M0);  // 0: a warp without tokens
-      const float f1 = (m1 == -INFINITY) ? 0.f : exp2f(m1 - M1);
+      const float f0 = (st.m0 == -INFINITY) ? 0.f : exp2f(st.m0 - M0);  // 0: a warp without tokens
+      const float f1 = (st.m1 == -INFINITY) ? 0.f : exp2f(st.m1 - M1);
 #pragma unroll
       for (int wq = 0; wq < kW; ++wq) {
         if (warp == wq) {
@@ -817,15 +729,15 @@ __global__ void __launch_bounds__(kT, 1) fused_layer_kernel(const LayerArgs a, c
             float* r0p = sO + (2 * t) * kOPitch + 16 * mt + g;
             float* r1p = sO + (2 * t + 1) * kOPitch + 16 * mt + g;
             if (wq == 0) {
-              r0p[0] = acc[mt][0] * f0;
-              r1p[0] = acc[mt][1] * f1;
-              r0p[8] = acc[mt][2] * f0;
-              r1p[8] = acc[mt][3] * f1;
+              r0p[0] = st.acc[mt][0] * f0;
+              r1p[0] = st.acc[mt][1] * f1;
+              r0p[8] = st.acc[mt][2] * f0;
+              r1p[8] = st.acc[mt][3] * f1;
             } else {
-              r0p[0] += acc[mt][0] * f0;
-              r1p[0] += acc[mt][1] * f1;
-              r0p[8] += acc[mt][2] * f0;
-              r1p[8] += acc[mt][3] * f1;
+              r0p[0] += st.acc[mt][0] * f0;
+              r1p[0] += st.acc[mt][1] * f1;
+              r0p[8] += st.acc[mt][2] * f0;
+              r1p[8] += st.acc[mt][3] * f1;
             }
           }
         }

@@ -126,6 +126,9 @@ constexpr int kRowBytes = 128 * 2;                       // one K or V row
 constexpr int kMaxAttendHeads = 1024;                    // B * Hkv per layer
 constexpr int kMaxSelSlots = kMaxAttendHeads;            // retrieval slots per layer
 constexpr int kMaxSelectCtasPerSm = 2;                   // resident selection CTAs per SM
+// 16-byte key loads a selection thread keeps in flight per batch (two batches are in flight;
+// 10 and 12 measured slower on the 1M-context step)
+constexpr int kScoreUnroll = 8;
 constexpr int kScoreCap = 16384;                         // scores a selection CTA keeps on chip
 constexpr int kHistCopies = 8;                           // copies of each slot's histogram
 size_t select_smem_bytes(int slots);

@@ -244,7 +244,7 @@ __device__ __forceinline__ void select_body(const LayerArgs& a, const Workspace&
       }
       const uint4* keys =
           reinterpret_cast<const uint4*>(a.k_idx + head * (size_t)a.max_ctx * kIdxDim);
-      constexpr int kPairs = kSelThreads / 2, kUnroll = 8;
+      constexpr int kPairs = kSelThreads / 2, kUnroll = kScoreUnroll;
       float mx = -INFINITY;
       uint4 kv[kUnroll], nx[kUnroll];
       auto load_batch = [&](uint4 (&dst)[kUnroll], int base) {
