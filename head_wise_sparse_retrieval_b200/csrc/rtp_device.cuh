@@ -176,6 +176,31 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
 __device__ __forceinline__ float bf16_lo(uint32_t v) { return __uint_as_float(v << 16); }
 __device__ __forceinline__ float bf16_hi(uint32_t v) { return __uint_as_float(v & 0xffff0000u); }
 
+// ---- indexer score arithmetic --------------------------------------------------------------
+//
+// fp16 x fp16 products are exact in fp32 (11-bit significands, no overflow or underflow), so
+// the fp32 sum of two products, rounded once, is fma(a0, b0, a1 * b1): mixed-precision FMAs
+// with fp16 operands give it without converting the operands. The -0 addend keeps a zero
+// product's sign, so the result equals __fadd_rn(__fmul_rn(a0, b0), __fmul_rn(a1, b1)).
+__device__ __forceinline__ float dot2_f16(uint32_t a2, uint32_t b2) {
+  float d;
+  asm("{\n\t.reg .f16 al, ah, bl, bh;\n\t.reg .f32 p;\n\t"
+      "mov.b32 {al, ah}, %1;\n\tmov.b32 {bl, bh}, %2;\n\t"
+      "fma.rn.f32.f16 p, ah, bh, 0f80000000;\n\t"
+      "fma.rn.f32.f16 %0, al, bl, p;\n\t}"
+      : "=f"(d)
+      : "r"(a2), "r"(b2));
+  return d;
+}
+
+// Sum of the 8 products of two fp16 8-vectors (16 bytes each) in the fixed order
+// ((p0 + p1) + (p2 + p3)) + ((p4 + p5) + (p6 + p7)), fp32.
+__device__ __forceinline__ float dot8_f16(const uint4& a, const uint4& b) {
+  const float s01 = dot2_f16(a.x, b.x), s23 = dot2_f16(a.y, b.y);
+  const float s45 = dot2_f16(a.z, b.z), s67 = dot2_f16(a.w, b.w);
+  return __fadd_rn(__fadd_rn(s01, s23), __fadd_rn(s45, s67));
+}
+
 // ---- the histogram bin of a scaled indexer score -------------------------------------------
 //
 // bin = clamp(256 + floor((s - s_max) * bin_scale), 0, 255), bin_scale = 256 / idx_range.

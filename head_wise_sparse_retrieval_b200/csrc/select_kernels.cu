@@ -222,65 +222,49 @@ __device__ __forceinline__ void select_body(const LayerArgs& a, const Workspace&
   const Scores<kFits> sc{s_scores, s_bins, w.scores, w.bins, (size_t)w.ld, t0, soff};
 
   // ---- phase 1: indexer scores of this CTA's range -----------------------------------------
+  // One thread per token: the 16 fp16 dims of the key arrive as two 16-byte loads, the score
+  // is (dot8(dims 0-7) + dot8(dims 8-15)) * scale with the products summed pairwise in fp32.
   if (active) {
     int s = upper_slot(soff, S, t0);
-    const int half = tid & 1, pair = tid >> 1;
     for (long long t = t0; t < t1; ++s) {
       const int n0 = (int)(t - soff[s]);
       const int n1 = (int)(min(t1, soff[s + 1]) - soff[s]);
       t = soff[s] + n1;
       const int b = s / a.nret, kvh = a.ret_kvh[s % a.nret];
       const size_t head = (size_t)b * a.Hkv + kvh;
-      float q[8];
-      {
-        const uint4 qv = *reinterpret_cast<const uint4*>(a.q_idx + head * kIdxDim + half * 8);
-        const __half2* h2 = reinterpret_cast<const __half2*>(&qv);
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          const float2 f = __half22float2(h2[i]);
-          q[2 * i] = f.x;
-          q[2 * i + 1] = f.y;
-        }
-      }
+      const uint4 qlo = *reinterpret_cast<const uint4*>(a.q_idx + head * kIdxDim);
+      const uint4 qhi = *reinterpret_cast<const uint4*>(a.q_idx + head * kIdxDim + 8);
       const uint4* keys =
           reinterpret_cast<const uint4*>(a.k_idx + head * (size_t)a.max_ctx * kIdxDim);
-      constexpr int kPairs = kSelThreads / 2, kUnroll = kScoreUnroll;
+      float* srow = sc.at(s, 0);  // kFits: the slot's scores in this CTA's shared memory
+      constexpr int kUnroll = kScoreUnroll / 2;  // tokens per thread per batch (two loads each)
       float mx = -INFINITY;
-      uint4 kv[kUnroll], nx[kUnroll];
-      auto load_batch = [&](uint4 (&dst)[kUnroll], int base) {
+      uint4 kv[2 * kUnroll], nx[2 * kUnroll];
+      auto load_batch = [&](uint4 (&dst)[2 * kUnroll], int base) {
 #pragma unroll
         for (int u = 0; u < kUnroll; ++u) {
-          const int n = base + u * kPairs + pair;
-          dst[u] = (n < n1) ? __ldcs(keys + 2 * (size_t)n + half) : make_uint4(0, 0, 0, 0);
+          const int n = base + u * kSelThreads + tid;
+          const bool in = n < n1;
+          dst[2 * u] = in ? __ldcs(keys + 2 * (size_t)n) : make_uint4(0, 0, 0, 0);
+          dst[2 * u + 1] = in ? __ldcs(keys + 2 * (size_t)n + 1) : make_uint4(0, 0, 0, 0);
         }
       };
       load_batch(kv, n0);
-      for (int base = n0; base < n1; base += kPairs * kUnroll) {
-        if (base + kPairs * kUnroll < n1) load_batch(nx, base + kPairs * kUnroll);  // prefetch
+      for (int base = n0; base < n1; base += kSelThreads * kUnroll) {
+        if (base + kSelThreads * kUnroll < n1) load_batch(nx, base + kSelThreads * kUnroll);
 #pragma unroll
         for (int u = 0; u < kUnroll; ++u) {
-          const int n = base + u * kPairs + pair;
-          const __half2* h2 = reinterpret_cast<const __half2*>(&kv[u]);
-          float p[8];
-#pragma unroll
-          for (int i = 0; i < 4; ++i) {
-            const float2 f = __half22float2(h2[i]);
-            p[2 * i] = __fmul_rn(q[2 * i], f.x);      // fp16 x fp16 products are exact in fp32
-            p[2 * i + 1] = __fmul_rn(q[2 * i + 1], f.y);
-          }
-          // pairwise sum: 8 products, then the partner lane's 8
-          const float s01 = __fadd_rn(p[0], p[1]), s23 = __fadd_rn(p[2], p[3]);
-          const float s45 = __fadd_rn(p[4], p[5]), s67 = __fadd_rn(p[6], p[7]);
-          const float part = __fadd_rn(__fadd_rn(s01, s23), __fadd_rn(s45, s67));
-          const float other = __shfl_xor_sync(0xffffffffu, part, 1);
-          const float sv = __fmul_rn(__fadd_rn(part, other), a.idx_scale);
+          const int n = base + u * kSelThreads + tid;
+          const float sv = __fmul_rn(__fadd_rn(dot8_f16(qlo, kv[2 * u]), dot8_f16(qhi, kv[2 * u + 1])),
+                                     a.idx_scale);
           if (n < n1) {
-            if (half == 0) *sc.at(s, n) = sv;
+            if (kFits) srow[n] = sv;
+            else *sc.at(s, n) = sv;
             mx = fmaxf(mx, sv);
           }
         }
 #pragma unroll
-        for (int u = 0; u < kUnroll; ++u) kv[u] = nx[u];
+        for (int u = 0; u < 2 * kUnroll; ++u) kv[u] = nx[u];
       }
       mx = block_max(mx, redf);
       if (tid == 0) atomicMax(w.smax_key + s, float_key(mx));
