@@ -230,6 +230,17 @@ def cpu_model() -> str:
     return "unknown"
 
 
+def attend_source_hash() -> str:
+    """Hash of the attention kernel's sources (the kernel and its tile step), to tell whether
+    the recorded ncu traffic still describes the kernel that runs."""
+    import hashlib
+    h = hashlib.sha256()
+    for f in ("attend_kernel.cu", "attend_tile.cuh"):
+        with open(os.path.join(ROOT, "head_wise_sparse_retrieval_b200", "csrc", f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
 def step_read_bytes(plan) -> int:
     """An upper bound of the bytes a step reads, from the shapes alone: every retrieval head's
     indexer keys and all of its N tokens, every local head's window set."""
@@ -305,7 +316,7 @@ def run_reference(args, plan, rank, world):
     import oracle
     from head_wise_sparse_retrieval_b200 import workloads as W
     dev = "cuda" if torch.cuda.is_available() else "cpu"
-    layers = cpu_sample_layers(plan, per_kind=1)
+    layers = cpu_sample_layers(plan)  # two of each kind: more one-head units than host threads
     threads = oracle.max_threads()
     layer_fn = lambda l: W.make_layer(plan, l, dev)
     full = oracle_step_bytes(plan, layer_fn)
@@ -548,9 +559,7 @@ def main():
                                     "per_launch_ms": per_ms, "algorithmic_bytes_per_launch": per_b,
                                     "achieved": gbs, "frac": gbs / hbm}
     traffic = None
-    import hashlib
-    src = os.path.join(ROOT, "head_wise_sparse_retrieval_b200", "csrc", "attend_kernel.cu")
-    if hashlib.sha256(open(src, "rb").read()).hexdigest()[:16] == ATTEND_NCU["source_sha256_16"]:
+    if attend_source_hash() == ATTEND_NCU["source_sha256_16"]:
         traffic = att_bytes_per_launch * ATTEND_NCU["traffic_bytes"] / ATTEND_NCU["algorithmic_bytes"]
 
     # the same step at other p (the 1M-context configuration sweeps p over 0.8 / 0.9 / 0.95)

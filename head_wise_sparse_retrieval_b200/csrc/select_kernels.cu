@@ -306,11 +306,16 @@ __device__ __forceinline__ void select_body(const LayerArgs& a, const Workspace&
         // Its tokens are summed in registers instead, then once per warp.
         unsigned long long m0 = 0ull;
         unsigned n0cnt = 0u;
+        // on chip, the slot's rows are plain offsets into shared memory (computed once here:
+        // the bin stores below would otherwise make the compiler reload the slot offsets)
+        const float* srow = sc.at(s, 0);
+        unsigned char* brow = sc.bin_at(s, 0);
 #pragma unroll 4
         for (int n = k0 + tid; n < k1; n += kSelThreads) {
-          const float v = *sc.at(s, n);
+          const float v = kFits ? srow[n] : *sc.at(s, n);
           const int bin = score_bin(v, s_max, a.bin_scale);
-          *sc.bin_at(s, n) = (unsigned char)bin;
+          if (kFits) brow[n] = (unsigned char)bin;
+          else *sc.bin_at(s, n) = (unsigned char)bin;
           const float wgt = expf(v - s_max);                          // in (0, 1]
           const unsigned long long fx = __float2ull_rn(wgt * 1099511627776.0f);  // * 2^40, exact
           if (bin == 0) {
@@ -402,6 +407,7 @@ __device__ __forceinline__ void select_body(const LayerArgs& a, const Workspace&
         w.sel_n[s] = (int)(soff[s + 1] - soff[s]);
       }
       int* out = w.sel_idx + (size_t)s * w.ld;
+      const unsigned char* brow = sc.bin_at(s, 0);  // on chip: the slot's bins in shared memory
       // ordered compaction: warp w takes 32 x kPerThread consecutive tokens of each round, one
       // ballot per 32; the warps' counts are scanned, then each warp writes its tokens in order
       constexpr int kWarpSpan = 32 * kPerThread;
@@ -412,7 +418,8 @@ __device__ __forceinline__ void select_body(const LayerArgs& a, const Workspace&
 #pragma unroll
         for (int k = 0; k < kPerThread; ++k) {
           const int n = wb + 32 * k + lane;
-          const int bin = *sc.bin_at(s, min(n, n1 - 1));  // in range: no branch around the load
+          const int nc = min(n, n1 - 1);  // in range: no branch around the load
+          const int bin = kFits ? brow[nc] : *sc.bin_at(s, nc);
           const bool f = n < n1 && bin >= bs;
           bal[k] = __ballot_sync(0xffffffffu, f);
           wcnt += __popc(bal[k]);

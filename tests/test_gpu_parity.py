@@ -437,3 +437,36 @@ def test_profiling_and_nvtx_do_not_change_results():
     assert all(ms > 0 for _, ms in launches)
     check_output(dense.cpu().numpy()[0, 0:8], oracle_head(li, 0, 0, False, 0.9, 8,
                                                           dense=True).out, "dense after profiling")
+
+
+@pytest.mark.slow
+def test_largest_context_with_tied_scores_selects_every_token():
+    """The largest cache a handle takes (max_ctx = 2^24 - 1) with a zero indexer query: every
+    score ties at s_max = 0, every token falls in bin 255 with mass 1, and the 64-bit sums of
+    2^-40 fixed-point masses reach (2^24 - 1) * 2^40, just below 2^64. A wrapped sum would move
+    b* off bin 255 and drop tokens. With a zero query as well the attention weights are
+    uniform, so the output is the mean of V over all tokens (computed here by torch in fp64)."""
+    N = (1 << 24) - 1
+    g = torch.Generator(device=DEV).manual_seed(77)
+    k = torch.randn((1, 1, N, 128), generator=g, device=DEV, dtype=torch.bfloat16)
+    v = torch.randn((1, 1, N, 128), generator=g, device=DEV, dtype=torch.bfloat16)
+    k_idx = torch.randn((1, 1, N, 16), generator=g, device=DEV, dtype=torch.float16)
+    q = torch.zeros((1, 8, 128), dtype=torch.bfloat16, device=DEV)
+    q_idx = torch.zeros((1, 1, 16), dtype=torch.float16, device=DEV)
+    seq = torch.tensor([N], dtype=torch.int32, device=DEV)
+    p = W.custom(batch=1, num_q_heads=8, num_kv_heads=1, seq_lens=[N], max_ctx=N,
+                 retrieval=[1], kinds=[[W.KIND_FLAT]], seed=77)
+    out = torch.full((1, 8, 128), float("nan"), dtype=torch.float32, device=DEV)
+    cnt = torch.full((1, 1), -1, dtype=torch.int32, device=DEV)
+    with make_handle(p) as h:
+        h.decode_step(0, rtp.Layer(q, q_idx, k, v, k_idx, seq), np.array([1], np.uint8), 0.9,
+                      out, cnt)
+        torch.cuda.synchronize()
+        assert h.device_status() == 0
+        bstar, s_max = h.threshold(0, 0)
+    assert int(cnt.item()) == N
+    assert (bstar, s_max) == (255, 0.0)
+    ref = v[0, 0].double().mean(dim=0).cpu().numpy()
+    got = out[0].cpu().numpy()
+    for g_ in range(8):
+        check_output(got[g_:g_ + 1], ref[None, :], f"mean of V, query head {g_}")

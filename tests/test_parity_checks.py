@@ -69,7 +69,7 @@ def test_kernel_arithmetic_passes_with_margin(flat_head):
 
 
 def test_own_set_output_isolates_a_differing_selection(flat_head):
-    """A selection that differs from the oracle's by edge tokens is judged on its own set: the
+    """A selection that differs from the oracle's by edge tokens is compared on its own set: the
     own-set O1 is the oracle's attention over exactly the positions given."""
     li, ho = flat_head
     sel = ho.sel[:-1]  # as if the GPU had left out one edge token
