@@ -385,7 +385,7 @@ __global__ void __launch_bounds__(kT, 1) fused_layer_kernel(const LayerArgs a, c
     };
     for (int i = 0; i < kRing - 1; ++i) issue_keys(i);
     int s_cur = 0, run = -1;
-    float q[8];
+    uint4 qv = make_uint4(0, 0, 0, 0);  // this lane's 8 fp16 dims of the slot's indexer query
     float mx = -INFINITY;
     auto flush_max = [&]() {
 #pragma unroll
@@ -403,15 +403,8 @@ __global__ void __launch_bounds__(kT, 1) fused_layer_kernel(const LayerArgs a, c
         run = s_cur;
         mx = -INFINITY;
         const int b = run / a.nret, kvh = a.ret_kvh[run % a.nret];
-        const uint4 qv = *reinterpret_cast<const uint4*>(
+        qv = *reinterpret_cast<const uint4*>(
             a.q_idx + ((size_t)b * a.Hkv + kvh) * kIdxDim + (lane & 1) * 8);
-        const __half2* h2 = reinterpret_cast<const __half2*>(&qv);
-#pragma unroll
-        for (int k = 0; k < 4; ++k) {
-          const float2 fq = __half22float2(h2[k]);
-          q[2 * k] = fq.x;
-          q[2 * k + 1] = fq.y;
-        }
       }
       const int valid = min(kOwn, tb.N[run] - tile_n0(o, run));
       const unsigned char* st = smem + (warp * kRing + i % kRing) * kKeyStage;
@@ -419,18 +412,9 @@ __global__ void __launch_bounds__(kT, 1) fused_layer_kernel(const LayerArgs a, c
       for (int pp = 0; pp < 4; ++pp) {
         const int tok = pp * 16 + (lane >> 1);
         const uint4 kv = *reinterpret_cast<const uint4*>(st + (tok * 2 + (lane & 1)) * 16);
-        const __half2* h2 = reinterpret_cast<const __half2*>(&kv);
-        float p[8];
-#pragma unroll
-        for (int k = 0; k < 4; ++k) {
-          const float2 fk = __half22float2(h2[k]);
-          p[2 * k] = __fmul_rn(q[2 * k], fk.x);  // fp16 x fp16 products are exact in fp32
-          p[2 * k + 1] = __fmul_rn(q[2 * k + 1], fk.y);
-        }
-        // pairwise sums in the selection kernel's order: 8 products, then the other half's 8
-        const float s01 = __fadd_rn(p[0], p[1]), s23 = __fadd_rn(p[2], p[3]);
-        const float s45 = __fadd_rn(p[4], p[5]), s67 = __fadd_rn(p[6], p[7]);
-        const float part = __fadd_rn(__fadd_rn(s01, s23), __fadd_rn(s45, s67));
+        // the selection kernel's arithmetic: this half's 8 exact products summed pairwise in
+        // fp32 (mixed-precision FMAs), then the other half's sum added
+        const float part = dot8_f16(qv, kv);
         const float other = __shfl_xor_sync(0xffffffffu, part, 1);
         const float sv = __fmul_rn(__fadd_rn(part, other), a.idx_scale);
         if (tok < valid) {
