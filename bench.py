@@ -256,6 +256,66 @@ def step_read_bytes(plan) -> int:
     return total
 
 
+def prefill_rows_read(plan, masks: dict, T: int, dense: bool) -> int:
+    """Key rows the prefill streams into shared memory for a T-token prompt: row i of a head
+    reads its whole set once (i + 1 rows, or at most window + sinks for a local head)."""
+    n = np.arange(1, T + 1, dtype=np.int64)
+    full = int(n.sum())
+    win = int(np.minimum(n, plan.window + plan.sinks).sum())
+    B, Hkv = plan.batch, plan.num_kv_heads
+    if dense:
+        return plan.num_layers * B * Hkv * full
+    rows = 0
+    for m, ls in masks.items():
+        nret = int(np.frombuffer(m, np.uint8).astype(bool).sum())
+        rows += len(ls) * B * (nret * full + (Hkv - nret) * win)
+    return rows
+
+
+def prefill_leg(h, plan, kcache, vcache, dev, stream, T: int) -> dict:
+    """A T-token prompt through every layer (rtp_prefill with the layer's retrieval mask), and the
+    same with every head dense (the kernel's full causal attention): one call per distinct mask,
+    timed with CUDA events on the launch stream after a warm-up call, summed over the layers."""
+    import torch
+    B, Hq, Hkv, L = plan.batch, plan.num_q_heads, plan.num_kv_heads, plan.num_layers
+    gen = torch.Generator(device=dev).manual_seed(7)
+    q = torch.randn(B, Hq, T, 128, generator=gen, device=dev).to(torch.bfloat16)
+    out = torch.empty(B, Hq, T, 128, dtype=torch.float32, device=dev)
+    seq = torch.full((B,), T, dtype=torch.int32, device=dev)
+    masks = {}
+    for l in range(L):
+        masks.setdefault(bytes(plan.retrieval[l].astype(np.uint8)), []).append(l)
+
+    def timed(mask, dense):
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        with torch.cuda.stream(stream):
+            h.prefill(q, kcache, vcache, seq, mask, out, dense=dense, stream=stream)
+            e0.record(stream)
+            h.prefill(q, kcache, vcache, seq, mask, out, dense=dense, stream=stream)
+            e1.record(stream)
+        torch.cuda.synchronize()
+        return e0.elapsed_time(e1)
+
+    per_mask = {m: timed(np.frombuffer(m, np.uint8).copy(), False) for m in masks}
+    sparse_ms = sum(per_mask[m] * len(ls) for m, ls in masks.items())
+    dense_ms = timed(np.zeros(Hkv, np.uint8), True) * L
+    rows_s = prefill_rows_read(plan, masks, T, False)
+    rows_d = prefill_rows_read(plan, masks, T, True)
+    flop_per_row = 2 * 2 * (Hq // Hkv) * 128  # S = K Q^T and O += V^T P^T, per query head
+    return {"prompt_tokens": T, "layers": L, "ms_sparse": sparse_ms, "ms_dense": dense_ms,
+            "speedup_vs_dense": dense_ms / sparse_ms,
+            "per_layer_ms": {"".join(str(x) for x in m): per_mask[m] for m in masks},
+            "smem_fill_tbs": {"sparse": rows_s * ROW_BYTES / (sparse_ms * 1e-3) / 1e12,
+                              "dense": rows_d * ROW_BYTES / (dense_ms * 1e-3) / 1e12},
+            "tflops": {"sparse": rows_s * flop_per_row / (sparse_ms * 1e-3) / 1e12,
+                       "dense": rows_d * flop_per_row / (dense_ms * 1e-3) / 1e12},
+            "kernel": "prefill_kernel",
+            "note": ("each row's key set is gathered from L2 into shared memory once per "
+                     "(row, KV head); the pages quote their prefill speed-up against "
+                     "FlashAttention-2 on H20 (2.83x at 32K), context only")}
+
+
 def config_of(plan, world: int) -> dict:
     """The workload both arms measure (the same keys and values for the GPU arm and the
     reference arm); how each arm times it is reported under "protocol"."""
@@ -366,6 +426,9 @@ def main():
     ap.add_argument("--k-sweep", default="2048,4096,16384",
                     help="fixed top-k values (through the same histogram) timed the same way")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-prefill", action="store_true")
+    ap.add_argument("--prefill-t", type=int, default=32768,
+                    help="prompt length of the prefill leg (the pages' prefill table starts at 32K)")
     ap.add_argument("--single-layer", type=int, default=None,
                     help="profiling case: only this layer of the workload, decoded --reps times")
     ap.add_argument("--reps", type=int, default=3)
@@ -647,6 +710,12 @@ def main():
                "shape": {"batch": B, "q_heads": Hq, "kv_heads": Hkv, "r": 16}}
     del gi, ki_s
 
+    # prefill of a prompt through every layer's mask, against dense prefill on the same kernel
+    prefill = None
+    if not args.no_prefill and args.prefill_t <= plan.max_ctx:
+        prefill = prefill_leg(h, plan, layers[0].k_cache, layers[0].v_cache, dev, stream,
+                              args.prefill_t)
+
     # dense decode on the same caches (the speedup denominator)
     dense = None
     if not args.no_dense:
@@ -757,6 +826,7 @@ def main():
         "chained": chained,
         "single_launch": single,
         "indexer_append": indexer,
+        "prefill": prefill,
         "dense": dense,
         "e2e": e2e,
         "cpu_baseline": cpu,

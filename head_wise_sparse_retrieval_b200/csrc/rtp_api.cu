@@ -32,6 +32,7 @@ struct rtp_handle {
   int fused_grid = 0;
   size_t fused_smem = 0;
   FusedArgs fx{};
+  int prefill_grid = 0;  // persistent prefill launch: every CTA resident at once
   // staging for rtp_decode_step_host
   void* stage_q = nullptr;
   void* stage_qidx = nullptr;
@@ -488,6 +489,21 @@ rtp_status rtp_create(const rtp_config* cfg, int device, rtp_handle** out) {
     }
     h->fused_ok = per_sm >= 1;  // the grid is one CTA per SM, all resident at once
   }
+  {  // prefill: a persistent grid of as many CTAs as fit at once (at most two per SM)
+    int per_sm = 0;
+    e = raise_smem_limit((const void*)prefill_kernel, prefill_smem_bytes());
+    if (e == cudaSuccess)
+      e = cudaFuncSetAttribute(prefill_kernel, cudaFuncAttributePreferredSharedMemoryCarveout, 100);
+    if (e == cudaSuccess)
+      e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, prefill_kernel,
+                                                        kPrefillWarps * 32, prefill_smem_bytes());
+    if (e != cudaSuccess) {
+      cudaFree(h->ws_mem);
+      delete h;
+      return cuda_fail(e, "cudaFuncSetAttribute(prefill_kernel)");
+    }
+    h->prefill_grid = h->num_sms * (per_sm < 2 ? per_sm : 2);
+  }
   *out = h;
   return ok();
 }
@@ -601,6 +617,58 @@ rtp_status rtp_selftest_wait_timeout(rtp_handle* h, int layer, const rtp_layer_i
   if (st != RTP_OK) return st;
   h->last_valid = false;  // its selection lists are not meaningful
   return ok();
+}
+
+rtp_status rtp_prefill(rtp_handle* h, const rtp_prefill_io* io, void* stream) {
+  if (!h) return fail(RTP_ERR_INVALID_ARG, "handle is NULL");
+  if (!io || !io->q || !io->k_cache || !io->v_cache || !io->seq_lens || !io->out ||
+      !io->retrieval_mask)
+    return fail(RTP_ERR_INVALID_ARG, "a required pointer is NULL");
+  if (!aligned16(io->q) || !aligned16(io->k_cache) || !aligned16(io->v_cache) ||
+      !aligned16(io->out) || ((uintptr_t)io->seq_lens & 3u))
+    return fail(RTP_ERR_INVALID_ARG, "pointers must be 16-byte aligned (seq_lens 4)");
+  if (io->t_max < 1 || io->t_max > h->cfg.max_ctx)
+    return fail(RTP_ERR_INVALID_ARG, "t_max %d outside [1, max_ctx = %d]", io->t_max,
+                h->cfg.max_ctx);
+  if ((long long)h->cfg.batch * h->cfg.num_kv_heads * io->t_max > 0x7fffffffLL)
+    return fail(RTP_ERR_UNSUPPORTED, "batch * num_kv_heads * t_max must be < 2^31");
+  if (h->prefill_grid < 1) return fail(RTP_ERR_UNSUPPORTED, "prefill_kernel does not fit an SM");
+  PrefillArgs a;
+  memset(&a, 0, sizeof a);
+  a.q = static_cast<const __nv_bfloat16*>(io->q);
+  a.k_cache = static_cast<const __nv_bfloat16*>(io->k_cache);
+  a.v_cache = static_cast<const __nv_bfloat16*>(io->v_cache);
+  a.seq_lens = io->seq_lens;
+  a.out = io->out;
+  a.status = h->ws.status;
+  a.B = h->cfg.batch;
+  a.Hq = h->cfg.num_q_heads;
+  a.Hkv = h->cfg.num_kv_heads;
+  a.G = h->G;
+  a.max_ctx = h->cfg.max_ctx;
+  a.t_max = io->t_max;
+  a.window = h->cfg.window;
+  a.sinks = h->cfg.sinks;
+  a.dense = io->dense ? 1 : 0;
+  a.attn_scale_log2 = (float)((double)h->cfg.attn_scale * 1.4426950408889634);
+  unsigned long long bits[4] = {0ull, 0ull, 0ull, 0ull};
+  for (int k = 0; k < a.Hkv; ++k)
+    if (io->retrieval_mask[k]) bits[k >> 6] |= 1ull << (k & 63);
+  a.ret_bits0 = bits[0];
+  a.ret_bits1 = bits[1];
+  a.ret_bits2 = bits[2];
+  a.ret_bits3 = bits[3];
+  const long long warps = (long long)a.B * a.Hkv * a.t_max;  // one warp per (b, KV head, row)
+  const long long need = (warps + kPrefillWarps - 1) / kPrefillWarps;
+  const int grid = need < h->prefill_grid ? (int)need : h->prefill_grid;
+  DeviceGuard guard(h->device);
+  NvtxRange range(h, "rtp_prefill (t_max %d, dense %d)", io->t_max, a.dense);
+  // a plain launch (no programmatic dependency): the kernel starts after the preceding work on
+  // the stream has completed
+  prefill_kernel<<<grid, kPrefillWarps * 32, prefill_smem_bytes(),
+                   static_cast<cudaStream_t>(stream)>>>(a);
+  const cudaError_t e = cudaGetLastError();
+  return e == cudaSuccess ? ok() : cuda_fail(e, "prefill_kernel launch");
 }
 
 rtp_status rtp_dense_decode(rtp_handle* h, const rtp_layer_io* io, void* stream) {

@@ -86,6 +86,25 @@ struct FusedArgs {
 __global__ void fused_layer_kernel(const LayerArgs a, const Workspace w, const FusedArgs f);
 size_t fused_smem_bytes();
 
+// Prefill (prefill_kernel.cu): attention of every position of a prompt, over all earlier
+// positions for retrieval heads (or every head, dense), over sinks + window for local heads.
+// Persistent grid; one warp per work item (b, KV head, row).
+constexpr int kPrefillWarps = 4;
+struct PrefillArgs {
+  const __nv_bfloat16* q;         // [B][Hq][t_max][128]
+  const __nv_bfloat16* k_cache;   // [B][Hkv][max_ctx][128], rows < T_b hold the prompt
+  const __nv_bfloat16* v_cache;
+  const int* seq_lens;            // [B] prompt lengths T_b
+  float* out;                     // [B][Hq][t_max][128]
+  unsigned* status;
+  // retrieval KV heads: bit kvh of the 256-bit mask
+  unsigned long long ret_bits0, ret_bits1, ret_bits2, ret_bits3;
+  int B, Hq, Hkv, G, max_ctx, t_max, window, sinks, dense;
+  float attn_scale_log2;
+};
+__global__ void prefill_kernel(const PrefillArgs a);
+size_t prefill_smem_bytes();
+
 // Indexer production at decode (indexer_kernel.cu).
 struct IndexerArgs {
   const __nv_bfloat16* q_pre;     // [B][Hq][128]

@@ -26,7 +26,7 @@ EXPORTS = ("rtp_config_default", "rtp_workspace_bytes", "rtp_create", "rtp_destr
            "rtp_get_threshold", "rtp_get_device_status", "rtp_status_string", "rtp_last_error",
            "rtp_profile_enable", "rtp_profile_read", "rtp_window_attention_noalloc",
            "rtp_indexer_append", "rtp_selftest_wait_timeout", "rtp_nvtx_enable",
-           "rtp_profile_launches")
+           "rtp_profile_launches", "rtp_prefill")
 NOALLOC_MAX_HEADS = 64
 KERNEL_CLASSES = ("select", "attend", "merge", "fused")
 
@@ -61,6 +61,14 @@ class IndexerIO(ctypes.Structure):
         ("w_k", ctypes.c_void_p), ("seq_lens", ctypes.c_void_p),
         ("head_mask", ctypes.POINTER(ctypes.c_uint8)), ("q_idx", ctypes.c_void_p),
         ("k_idx", ctypes.c_void_p),
+    ]
+
+
+class PrefillIO(ctypes.Structure):
+    _fields_ = [
+        ("q", ctypes.c_void_p), ("k_cache", ctypes.c_void_p), ("v_cache", ctypes.c_void_p),
+        ("seq_lens", ctypes.c_void_p), ("retrieval_mask", ctypes.POINTER(ctypes.c_uint8)),
+        ("out", ctypes.c_void_p), ("t_max", ctypes.c_int32), ("dense", ctypes.c_int32),
     ]
 
 
@@ -114,6 +122,8 @@ def load(path: str = LIB_PATH):
     L.rtp_window_attention_noalloc.restype = ctypes.c_int
     L.rtp_indexer_append.argtypes = [vp, ctypes.POINTER(IndexerIO), vp]
     L.rtp_indexer_append.restype = ctypes.c_int
+    L.rtp_prefill.argtypes = [vp, ctypes.POINTER(PrefillIO), vp]
+    L.rtp_prefill.restype = ctypes.c_int
     L.rtp_selftest_wait_timeout.argtypes = [vp, i, ctypes.POINTER(LayerIO), ctypes.c_uint64, vp]
     L.rtp_selftest_wait_timeout.restype = ctypes.c_int
     L.rtp_status_string.argtypes = [i]
@@ -251,6 +261,17 @@ class Handle:
         _check(load().rtp_indexer_append(self._h, ctypes.byref(io), _stream_ptr(stream)),
                "rtp_indexer_append")
 
+    def prefill(self, q, k_cache, v_cache, seq_lens, mask, out, dense: bool = False,
+                stream=None):
+        """rtp_prefill: q [B, Hq, t_max, 128] bf16 -> out [B, Hq, t_max, 128] fp32 (rows below
+        each prompt length), over caches whose rows 0 .. T_b - 1 hold the prompt."""
+        m = np.ascontiguousarray(np.asarray(mask, dtype=np.uint8))
+        assert m.shape == (self.cfg.num_kv_heads,)
+        io = PrefillIO(_ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(seq_lens),
+                       m.ctypes.data_as(ctypes.POINTER(ctypes.c_uint8)), _ptr(out),
+                       int(q.shape[2]), 1 if dense else 0)
+        _check(load().rtp_prefill(self._h, ctypes.byref(io), _stream_ptr(stream)), "rtp_prefill")
+
     def selftest_wait_timeout(self, layer_idx: int, layer: Layer, mask, top_p: float, out,
                               wait_ns: int, stream=None):
         """rtp_selftest_wait_timeout: the layer's selection with one barrier arrival withheld."""
@@ -297,7 +318,7 @@ class Handle:
         kind = (ctypes.c_int32 * cap)()
         n = ctypes.c_int64()
         _check(load().rtp_profile_launches(self._h, ms, kind, cap, ctypes.byref(n)),
-               "rtp_profile_launches")
+               "rtp_profile_launches", "rtp_prefill")
         return [(KERNEL_CLASSES[kind[i]], ms[i]) for i in range(n.value)]
 
     def device_status(self) -> int:

@@ -179,6 +179,36 @@ typedef struct {
 
 RTP_API rtp_status rtp_indexer_append(rtp_handle *h, const rtp_indexer_io *io, void *stream);
 
+/* ---- Prefill ---------------------------------------------------------------------------
+ * gist.science technical summary, Methodology 1: during prefill the retrieval heads keep, and
+ * attend over, the full KV cache, and the local heads a sliding window with attention sinks;
+ * "Full Attention Strikes Back ..." (xllm-io paper review) section 五 测试配置 (window 8192,
+ * 4 sinks) and its prefill speed-up table. For every prompt position i < T_b of sequence b and
+ * every query head hq of KV head kvh = hq / G:
+ *   out[b][hq][i] = sum_{j in K_i} softmax_{K_i}(attn_scale * q[b][hq][i] . k_j) v_j
+ *   K_i = { j : j <= i }                                          retrieval head, or dense != 0
+ *   K_i = { 0 .. sinks-1 } U { i+1-window .. i } (all j <= i when they meet)   local head
+ * i.e. the decode output of a context of i + 1 tokens (window and sinks from the config). The
+ * caller has written the prompt's keys and values into rows 0 .. T_b - 1 of the caches. Rows
+ * i >= T_b of out are not written. One launch, no host synchronisation, no allocation; the
+ * kernel starts once the preceding work on the stream has completed. Errors (nothing
+ * enqueued): RTP_ERR_INVALID_ARG for a NULL / misaligned pointer or t_max outside
+ * [1, max_ctx]; RTP_ERR_UNSUPPORTED for batch * num_kv_heads * t_max >= 2^31. A seq_lens entry
+ * outside [1, t_max] is clamped and reported in the device status word. */
+typedef struct {
+    const void *q;           /* bf16 [B][Hq][t_max][D], device: the prompt's queries           */
+    const void *k_cache;     /* bf16 [B][Hkv][max_ctx][D], device                              */
+    const void *v_cache;     /* bf16 [B][Hkv][max_ctx][D], device                              */
+    const int32_t *seq_lens; /* [B], device: prompt lengths T_b                                */
+    const uint8_t *retrieval_mask; /* [Hkv], HOST: nonzero marks a retrieval KV head           */
+    float *out;              /* fp32 [B][Hq][t_max][D], device: rows < T_b written             */
+    int32_t t_max;           /* rows per head of q and out, 1 .. max_ctx                      */
+    int32_t dense;           /* nonzero: every head attends over all j <= i (full causal
+                                attention, the speed-up denominator)                          */
+} rtp_prefill_io;
+
+RTP_API rtp_status rtp_prefill(rtp_handle *h, const rtp_prefill_io *io, void *stream);
+
 /* Dense full attention over all N_b tokens for every KV head (top_p, q_idx, k_idx and the mask
  * are ignored). The speedup denominator: same caches, same kernels, no selection. */
 RTP_API rtp_status rtp_dense_decode(rtp_handle *h, const rtp_layer_io *io, void *stream);

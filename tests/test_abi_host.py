@@ -91,6 +91,8 @@ def test_calls_on_null_handle_are_rejected(rtp_lib):
     n = ctypes.c_int64()
     assert L.rtp_profile_launches(None, None, None, 0, ctypes.byref(n)) == \
         rtp_lib.RTP_ERR_INVALID_ARG
+    pio = rtp_lib.PrefillIO()
+    assert L.rtp_prefill(None, ctypes.byref(pio), None) == rtp_lib.RTP_ERR_INVALID_ARG
     assert L.rtp_destroy(None) == rtp_lib.RTP_OK
     assert L.rtp_status_string(3) == b"RTP_ERR_OOM"
 
