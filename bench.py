@@ -256,20 +256,27 @@ def step_read_bytes(plan) -> int:
     return total
 
 
-def prefill_rows_read(plan, masks: dict, T: int, dense: bool) -> int:
-    """Key rows the prefill streams into shared memory for a T-token prompt: row i of a head
-    reads its whole set once (i + 1 rows, or at most window + sinks for a local head)."""
+def prefill_key_counts(plan, masks: dict, T: int, dense: bool) -> tuple[int, int]:
+    """(rows, fills) of a T-token prompt through every layer: rows = the sum over prompt rows of
+    their key-set sizes (i + 1, or at most window + sinks for a local head): the attention's
+    work; fills = the key rows gathered into shared memory, one union set per pair of rows."""
+    W, S = plan.window, plan.sinks
     n = np.arange(1, T + 1, dtype=np.int64)
-    full = int(n.sum())
-    win = int(np.minimum(n, plan.window + plan.sinks).sum())
+    rows_full, rows_win = int(n.sum()), int(np.minimum(n, W + S).sum())
+    lo = np.arange(0, T, 2, dtype=np.int64)
+    hi = np.minimum(lo + 1, T - 1)
+    fill_full = int((hi + 1).sum())
+    fill_win = int(np.where(lo + 1 > W + S, S + W + (hi - lo), hi + 1).sum())
     B, Hkv = plan.batch, plan.num_kv_heads
     if dense:
-        return plan.num_layers * B * Hkv * full
-    rows = 0
+        k = plan.num_layers * B * Hkv
+        return k * rows_full, k * fill_full
+    rows = fills = 0
     for m, ls in masks.items():
         nret = int(np.frombuffer(m, np.uint8).astype(bool).sum())
-        rows += len(ls) * B * (nret * full + (Hkv - nret) * win)
-    return rows
+        rows += len(ls) * B * (nret * rows_full + (Hkv - nret) * rows_win)
+        fills += len(ls) * B * (nret * fill_full + (Hkv - nret) * fill_win)
+    return rows, fills
 
 
 def prefill_leg(h, plan, kcache, vcache, dev, stream, T: int) -> dict:
@@ -300,20 +307,20 @@ def prefill_leg(h, plan, kcache, vcache, dev, stream, T: int) -> dict:
     per_mask = {m: timed(np.frombuffer(m, np.uint8).copy(), False) for m in masks}
     sparse_ms = sum(per_mask[m] * len(ls) for m, ls in masks.items())
     dense_ms = timed(np.zeros(Hkv, np.uint8), True) * L
-    rows_s = prefill_rows_read(plan, masks, T, False)
-    rows_d = prefill_rows_read(plan, masks, T, True)
+    rows_s, fills_s = prefill_key_counts(plan, masks, T, False)
+    rows_d, fills_d = prefill_key_counts(plan, masks, T, True)
     flop_per_row = 2 * 2 * (Hq // Hkv) * 128  # S = K Q^T and O += V^T P^T, per query head
     return {"prompt_tokens": T, "layers": L, "ms_sparse": sparse_ms, "ms_dense": dense_ms,
             "speedup_vs_dense": dense_ms / sparse_ms,
             "per_layer_ms": {"".join(str(x) for x in m): per_mask[m] for m in masks},
-            "smem_fill_tbs": {"sparse": rows_s * ROW_BYTES / (sparse_ms * 1e-3) / 1e12,
-                              "dense": rows_d * ROW_BYTES / (dense_ms * 1e-3) / 1e12},
+            "smem_fill_tbs": {"sparse": fills_s * ROW_BYTES / (sparse_ms * 1e-3) / 1e12,
+                              "dense": fills_d * ROW_BYTES / (dense_ms * 1e-3) / 1e12},
             "tflops": {"sparse": rows_s * flop_per_row / (sparse_ms * 1e-3) / 1e12,
                        "dense": rows_d * flop_per_row / (dense_ms * 1e-3) / 1e12},
             "kernel": "prefill_kernel",
-            "note": ("each row's key set is gathered from L2 into shared memory once per "
-                     "(row, KV head); the pages quote their prefill speed-up against "
-                     "FlashAttention-2 on H20 (2.83x at 32K), context only")}
+            "note": ("each pair of prompt rows gathers the union of its key sets from L2 into "
+                     "shared memory once per KV head; the pages quote their prefill speed-up "
+                     "against FlashAttention-2 on H20 (2.83x at 32K), context only")}
 
 
 def config_of(plan, world: int) -> dict:

@@ -658,7 +658,8 @@ rtp_status rtp_prefill(rtp_handle* h, const rtp_prefill_io* io, void* stream) {
   a.ret_bits1 = bits[1];
   a.ret_bits2 = bits[2];
   a.ret_bits3 = bits[3];
-  const long long warps = (long long)a.B * a.Hkv * a.t_max;  // one warp per (b, KV head, row)
+  // one warp per (b, KV head, pair of rows)
+  const long long warps = (long long)a.B * a.Hkv * ((a.t_max + 1) / 2);
   const long long need = (warps + kPrefillWarps - 1) / kPrefillWarps;
   const int grid = need < h->prefill_grid ? (int)need : h->prefill_grid;
   DeviceGuard guard(h->device);

@@ -318,7 +318,7 @@ class Handle:
         kind = (ctypes.c_int32 * cap)()
         n = ctypes.c_int64()
         _check(load().rtp_profile_launches(self._h, ms, kind, cap, ctypes.byref(n)),
-               "rtp_profile_launches", "rtp_prefill")
+               "rtp_profile_launches")
         return [(KERNEL_CLASSES[kind[i]], ms[i]) for i in range(n.value)]
 
     def device_status(self) -> int:
