@@ -441,6 +441,10 @@ def main():
     ap.add_argument("--reps", type=int, default=3)
     ap.add_argument("--single-launch", action="store_true",
                     help="--single-layer: run the layer as one fused launch")
+    ap.add_argument("--prefill-case", type=int, default=None,
+                    help="profiling case: rtp_prefill of a prompt of this many tokens with the "
+                         "mask of the workload's first layer that has a retrieval head, --reps "
+                         "calls")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
 
@@ -464,6 +468,28 @@ def main():
 
     rtp.load()
     dev = torch.device("cuda", local if world > 1 else 0)
+    if args.prefill_case is not None:  # small case for ncu captures of the prefill kernel
+        T = args.prefill_case
+        B, Hq, Hkv = plan.batch, plan.num_q_heads, plan.num_kv_heads
+        l = next(i for i in range(plan.num_layers) if plan.retrieval[i].any())
+        gen = torch.Generator(device=dev).manual_seed(T)
+        q = torch.randn(B, Hq, T, 128, generator=gen, device=dev).to(torch.bfloat16)
+        k = torch.randn(B, Hkv, T, 128, generator=gen, device=dev).to(torch.bfloat16)
+        v = torch.randn(B, Hkv, T, 128, generator=gen, device=dev).to(torch.bfloat16)
+        seq = torch.full((B,), T, dtype=torch.int32, device=dev)
+        out = torch.empty(B, Hq, T, 128, dtype=torch.float32, device=dev)
+        h = rtp.Handle(rtp.config_for(plan, max_ctx=T), dev.index)
+        for _ in range(args.reps):
+            h.prefill(q, k, v, seq, plan.retrieval[l], out)
+        torch.cuda.synchronize()
+        status = h.device_status()
+        h.close()
+        print(json.dumps({"prefill_case": T, "workload": plan.name, "mask_of_layer": l,
+                          "retrieval": plan.retrieval[l].tolist(), "reps": args.reps,
+                          "device_status": status}))
+        if status:
+            raise SystemExit(1)
+        return
     if args.single_layer is not None:  # small case for ncu captures (one layer, a few calls)
         l = args.single_layer
         li = W.make_layer(plan, l, dev)

@@ -11,7 +11,7 @@
 //
 // Work item = (b, KV head, rows 2p and 2p + 1): two decode problems whose token sets differ in
 // at most two positions, attended by one warp over the union of the two sets with the decode
-// attention's gather (attend_tile.cuh): 16-token tiles from the warp's own 3-stage cp.async
+// attention's gather (attend_tile.cuh): 16-token tiles from the warp's own 2-stage cp.async
 // pipeline. Each tile's K and V fragments are loaded from shared memory once and used by both
 // rows: S^T = K Q^T on the tensor cores with the G query heads of the group as N = 8, per row;
 // each row masks the tokens outside its own set, keeps its own online softmax (log2 domain) and
@@ -28,7 +28,7 @@ namespace {
 
 constexpr int kPW = kPrefillWarps;
 constexpr int kPT = kPW * 32;
-constexpr int kPDepth = 3;  // cp.async stages per warp
+constexpr int kPDepth = 2;  // cp.async stages per warp (12 warps per SM hide the latency)
 
 // B operand of the S MMA for row i: b0 = q[g][16 ks + 2t, +1], b1 = q[g][16 ks + 8 + 2t, +1] for
 // query head g = lane / 4 < G of the group (zeros above). Rows of one head are t_max apart.
@@ -138,7 +138,8 @@ __device__ __forceinline__ void prefill_tile2(uint32_t kb, const uint32_t (&qf)[
 size_t prefill_smem_bytes() { return (size_t)kPW * kPDepth * kWarpStage; }
 
 // The bound of 3 CTAs per SM caps the registers at 170 (the two rows' accumulators and queries
-// stay in registers; a few item-level values spill); shared memory admits two CTAs per SM.
+// stay in registers; a few item-level values spill); 64 KB of stages per CTA admit three CTAs
+// per SM in shared memory as well.
 __global__ void __launch_bounds__(kPT, 3) prefill_kernel(const PrefillArgs a) {
   extern __shared__ __align__(128) unsigned char smem[];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;

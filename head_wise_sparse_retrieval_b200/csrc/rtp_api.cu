@@ -489,7 +489,7 @@ rtp_status rtp_create(const rtp_config* cfg, int device, rtp_handle** out) {
     }
     h->fused_ok = per_sm >= 1;  // the grid is one CTA per SM, all resident at once
   }
-  {  // prefill: a persistent grid of as many CTAs as fit at once (at most two per SM)
+  {  // prefill: a persistent grid of as many CTAs as fit at once (at most three per SM)
     int per_sm = 0;
     e = raise_smem_limit((const void*)prefill_kernel, prefill_smem_bytes());
     if (e == cudaSuccess)
@@ -502,7 +502,7 @@ rtp_status rtp_create(const rtp_config* cfg, int device, rtp_handle** out) {
       delete h;
       return cuda_fail(e, "cudaFuncSetAttribute(prefill_kernel)");
     }
-    h->prefill_grid = h->num_sms * (per_sm < 2 ? per_sm : 2);
+    h->prefill_grid = h->num_sms * (per_sm < 3 ? per_sm : 3);
   }
   *out = h;
   return ok();
