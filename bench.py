@@ -602,15 +602,21 @@ def main():
     for _ in range(prof_steps):
         with torch.cuda.stream(stream):
             step()
-        launches = h.profile_launches()  # in launch order: [select,] attend, merge per layer
+        # in launch order, per layer: [select,] attend[, merge] (a layer of local heads only is
+        # one attention launch that merges inside, when the handle has its cluster size)
+        launches = h.profile_launches()
         at = 0
         for l in range(L):
             c = by_class.setdefault(layer_class(l), {"attend_ms": 0.0, "attend_n": 0,
                                                      "attend_bytes": 0, "select_ms": 0.0,
                                                      "select_n": 0, "select_bytes": 0})
+            seen_attend = False
             while at < len(launches):
                 kind, t_ms = launches[at]
+                if seen_attend and kind != "merge":
+                    break  # the next layer's first launch
                 at += 1
+                seen_attend = seen_attend or kind in ("attend", "fused")
                 acc[kind][0] += t_ms
                 acc[kind][1] += 1
                 if kind == "select":

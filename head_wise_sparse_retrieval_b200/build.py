@@ -8,7 +8,7 @@ ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 LIB = os.path.join(PKG, "librtp.so")
 SOURCES = ["rtp_api.cu", "select_kernels.cu", "attend_kernel.cu", "noalloc.cu",
-           "indexer_kernel.cu", "fused_kernel.cu", "prefill_kernel.cu"]
+           "indexer_kernel.cu", "fused_kernel.cu", "prefill_kernel.cu", "cluster_kernel.cu"]
 HEADERS = ["rtp_device.cuh", "rtp_kernels.h", "attend_tile.cuh"]
 NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")
 FLAGS = ["-gencode", "arch=compute_100a,code=sm_100a", "-O3", "-lineinfo", "-std=c++17",

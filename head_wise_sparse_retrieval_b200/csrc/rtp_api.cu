@@ -33,6 +33,9 @@ struct rtp_handle {
   size_t fused_smem = 0;
   FusedArgs fx{};
   int prefill_grid = 0;  // persistent prefill launch: every CTA resident at once
+  // layers without retrieval heads: one cluster of cluster_size CTAs per (b, KV head), or 0
+  int cluster_size = 0;
+  size_t cluster_smem = 0;
   // staging for rtp_decode_step_host
   void* stage_q = nullptr;
   void* stage_qidx = nullptr;
@@ -265,9 +268,41 @@ rtp_status enqueue_fused(rtp_handle* h, const LayerArgs& a, cudaStream_t s, int 
   return e == cudaSuccess ? RTP_OK : cuda_fail(e, "fused_layer_kernel launch");
 }
 
+// A launch of head_cluster_kernel: one cluster of h->cluster_size CTAs per (b, KV head), with
+// the programmatic-dependent-launch attribute of the other launches.
+cudaError_t launch_cluster(rtp_handle* h, const LayerArgs& a, cudaStream_t s) {
+  const bool prof = h->prof && h->prof_used < kProfCapacity;
+  if (h->prof && !prof) h->prof_overflow = true;
+  if (prof) cudaEventRecord(h->prof_ev[2 * h->prof_used], s);
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)(a.B * a.Hkv * h->cluster_size));
+  cfg.blockDim = dim3(kClusterWarps * 32);
+  cfg.dynamicSmemBytes = h->cluster_smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[2];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  attr[1].id = cudaLaunchAttributeClusterDimension;
+  attr[1].val.clusterDim.x = (unsigned)h->cluster_size;
+  attr[1].val.clusterDim.y = 1;
+  attr[1].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 2;
+  const cudaError_t e = cudaLaunchKernelEx(&cfg, head_cluster_kernel, a, h->ws);
+  if (prof && e == cudaSuccess) {
+    cudaEventRecord(h->prof_ev[2 * h->prof_used + 1], s);
+    h->prof_kind[h->prof_used++] = 1;  // an attention launch (its merge is inside)
+  }
+  return e;
+}
+
 rtp_status enqueue_layer(rtp_handle* h, const LayerArgs& a0, cudaStream_t s, int top_k = 0,
                          unsigned long long wait_ns = kWaitLimitNs, int withhold_cta = -1) {
   cudaError_t e;
+  if (!a0.dense && a0.nret == 0 && h->cluster_size > 0) {  // local heads only: one launch
+    e = launch_cluster(h, a0, s);
+    return e == cudaSuccess ? RTP_OK : cuda_fail(e, "head_cluster_kernel launch");
+  }
   if (!a0.dense && a0.nret > 0) {
     SelectArgs x;
     x.top_k = top_k;
@@ -488,6 +523,49 @@ rtp_status rtp_create(const rtp_config* cfg, int device, rtp_handle** out) {
       return cuda_fail(e, "cudaFuncSetAttribute(fused_layer_kernel)");
     }
     h->fused_ok = per_sm >= 1;  // the grid is one CTA per SM, all resident at once
+  }
+  {  // layers of local heads only: the largest cluster (kMinCluster .. kMaxCluster CTAs, one
+     // per SM) of which B * Hkv fit at once (else the largest of which one fits), when the SMs
+     // are enough for B * Hkv such clusters
+    const int nheads = cfg->batch * cfg->num_kv_heads;
+    int c = h->num_sms / nheads;
+    if (c > kMaxCluster) c = kMaxCluster;
+    h->cluster_smem = cluster_smem_bytes();
+    if (c >= kMinCluster && cfg->window + cfg->sinks <= kClusterMaxSet &&
+        h->cluster_smem <= (size_t)max_optin) {
+      e = raise_smem_limit((const void*)head_cluster_kernel, h->cluster_smem);
+      if (e == cudaSuccess)
+        e = cudaFuncSetAttribute(head_cluster_kernel,
+                                 cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+      for (; e == cudaSuccess && c >= kMinCluster; --c) {
+        cudaLaunchConfig_t lc = {};
+        lc.gridDim = dim3((unsigned)(nheads * c));
+        lc.blockDim = dim3(kClusterWarps * 32);
+        lc.dynamicSmemBytes = h->cluster_smem;
+        cudaLaunchAttribute at;
+        at.id = cudaLaunchAttributeClusterDimension;
+        at.val.clusterDim.x = (unsigned)c;
+        at.val.clusterDim.y = 1;
+        at.val.clusterDim.z = 1;
+        lc.attrs = &at;
+        lc.numAttrs = 1;
+        int nclusters = 0;
+        if (cudaOccupancyMaxActiveClusters(&nclusters, head_cluster_kernel, &lc) != cudaSuccess) {
+          cudaGetLastError();  // an unsupported size: try a smaller one
+          continue;
+        }
+        if (nclusters >= 1 && h->cluster_size == 0) h->cluster_size = c;  // the largest that fits
+        if (nclusters >= nheads) {  // one wave
+          h->cluster_size = c;
+          break;
+        }
+      }
+      if (e != cudaSuccess) {
+        cudaFree(h->ws_mem);
+        delete h;
+        return cuda_fail(e, "cudaFuncSetAttribute(head_cluster_kernel)");
+      }
+    }
   }
   {  // prefill: a persistent grid of as many CTAs as fit at once (at most three per SM)
     int per_sm = 0;

@@ -86,6 +86,17 @@ struct FusedArgs {
 __global__ void fused_layer_kernel(const LayerArgs a, const Workspace w, const FusedArgs f);
 size_t fused_smem_bytes();
 
+// Layers whose KV heads are all local heads (cluster_kernel.cu): one thread-block cluster of
+// up to kMaxCluster CTAs (one per SM) per (b, KV head), its pieces merged through distributed
+// shared memory.
+constexpr int kClusterWarps = 8;
+constexpr int kClusterDepth = 3;                         // cp.async stages per warp
+constexpr int kMaxCluster = 16;                          // CTAs of one cluster (non-portable > 8)
+constexpr int kMinCluster = 4;                           // below this the split launches serve better
+constexpr int kClusterMaxSet = 65536;                    // window + sinks of a cluster layer
+__global__ void head_cluster_kernel(const LayerArgs a, const Workspace w);
+size_t cluster_smem_bytes();
+
 // Prefill (prefill_kernel.cu): attention of every position of a prompt, over all earlier
 // positions for retrieval heads (or every head, dense), over sinks + window for local heads.
 // Persistent grid; one warp per work item (b, KV head, row).

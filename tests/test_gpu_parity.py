@@ -120,6 +120,40 @@ def test_small_window_and_no_sinks():
     _run(p, window=777, sinks=0)
 
 
+@pytest.mark.parametrize("B,Hkv,G,seq_lens", [
+    (1, 1, 8, [9000]),                       # one head: the most clusters per head
+    (1, 2, 8, [8197]),                       # two heads, window + sinks + 1 tokens
+    (1, 4, 8, [20000]),                      # the ctx_1m head layout
+    (2, 4, 4, [8196, 70]),                   # the whole context at and under window + sinks
+    (3, 4, 8, [1, 17, 12001]),               # 12 heads; contexts shorter than the cluster
+    (37, 1, 2, [3 + 331 * b for b in range(37)]),  # 37 heads: the smallest cluster
+    (40, 1, 1, [5000] * 40),                 # more heads than that serves: the split launches
+])
+def test_local_only_layers(B, Hkv, G, seq_lens):
+    """Layers without retrieval heads run as one launch of one or more thread-block clusters
+    per KV head when the SMs allow (their pieces merged in distributed shared memory, and across
+    clusters by a last-arriver ticket), else as the split attention and merge launches; every
+    head against the oracle, with the cache past each context poisoned, bit-identical reruns,
+    and the launch count of the path that ran."""
+    p = W.custom(batch=B, num_q_heads=Hkv * G, num_kv_heads=Hkv, seq_lens=seq_lens,
+                 max_ctx=max(seq_lens) + 5, retrieval=[0] * Hkv, kinds=[[0] * Hkv] * B,
+                 seed=B * 10 + Hkv)
+    li = W.make_layer(p, 0, DEV, poison_tail=True)
+    with make_handle(p) as h:
+        h.profile(True)
+        check_layer(h, p, li, 0)
+        kinds = [k for k, _ in h.profile_launches()]
+        h.profile(False)
+        a, _ = run_layer(h, p, li, 0)
+        b, _ = run_layer(h, p, li, 0)
+    assert torch.equal(a, b)
+    sms = torch.cuda.get_device_properties(0).multi_processor_count
+    if sms // (B * Hkv) >= 4:
+        assert kinds == ["attend"], kinds  # the merge is inside the launch
+    else:
+        assert kinds == ["attend", "merge"], kinds
+
+
 def test_all_retrieval_heads():
     p = W.custom(batch=2, num_q_heads=32, num_kv_heads=4, seq_lens=[40000, 25000],
                  max_ctx=40000, retrieval=[1, 1, 1, 1],
