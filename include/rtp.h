@@ -143,8 +143,12 @@ typedef struct {
                                 ignored (the launch always waits for the preceding one).          */
 } rtp_layer_io;
 
-/* Enqueues one layer of the decode step on `stream` (two kernels when the layer has retrieval
- * heads: the selection, then the attention of every head). Asynchronous: no host synchronisation,
+/* Enqueues one layer of the decode step on `stream`. A layer with retrieval heads is three
+ * kernels: the selection, the attention of every head (split over the SMs), and the merge of
+ * the split heads. A layer of local heads only is one kernel when the handle's B * Hkv leaves at
+ * least 4 SMs per KV head (and window + sinks <= 65536): one thread-block cluster per KV head,
+ * whose CTAs merge the head's pieces in distributed shared memory; otherwise attention and
+ * merge as above. Asynchronous: no host synchronisation,
  * no allocation, capturable in a CUDA graph (the mask is read on the host at call time and the
  * launch shapes depend only on cfg and the mask). Errors (nothing enqueued): RTP_ERR_INVALID_ARG
  * for a NULL handle / io / required pointer, a misaligned device pointer, top_k < 0, top_p
@@ -246,7 +250,8 @@ RTP_API rtp_status rtp_get_threshold(rtp_handle *h, int b, int kvh, int *bstar, 
  * launches on this handle is bracketed by two CUDA events recorded on the launch stream (the
  * events are created here, so the decode calls still allocate nothing). Do not enable it while
  * capturing a CUDA graph. Kernel classes: 0 selection (indexer score, histogram top-p,
- * compaction), 1 attention, 2 merge of split heads' partials, 3 the single-launch layer
+ * compaction), 1 attention (including the cluster launch of a layer of local heads only, which
+ * merges inside), 2 merge of split heads' partials, 3 the single-launch layer
  * (rtp_layer_io.single_launch). The event pool holds 1024
  * launches; rtp_profile_read empties it. Errors: RTP_ERR_CUDA if the events cannot be created. */
 RTP_API rtp_status rtp_profile_enable(rtp_handle *h, int enable);
