@@ -63,6 +63,81 @@ __device__ __forceinline__ int head_len(const LayerArgs& a, const Workspace& w, 
   return window_len(N, a.window, a.sinks);
 }
 
+// How a layer's heads are cut over the attention grid, from their token-set sizes. A head of
+// at most kTinyLen tokens (a concentrated query's few selected positions) takes a CTA of its
+// own when such heads are few (at most grid / 8, and the others keep a token per CTA):
+// otherwise the CTA holding it would also hold pieces of its neighbours and run an end-of-piece
+// merge for each. The other heads' sets are laid end to end (the tiny heads with no tokens) and
+// cut into P equal ranges, CTAs 0 .. P-1; the tiny heads follow in head order, CTAs P .. P +
+// ntiny - 1, each a single piece. Without such heads, or with too many, every set is laid end
+// to end (ntiny = 0). One warp calls it: off[1 .. nheads] hold the sizes on entry and the
+// inclusive scan of the laid-out sizes on return (off[0] = 0); every lane returns the same
+// values, including the head and size of CTA cta when it is a tiny head's (else -1, 0).
+constexpr int kTinyLen = 4 * kTile;
+struct HeadSplit {
+  long long T, P;   // laid-out tokens, CTAs that cut them
+  int ntiny;        // heads with a CTA of their own
+  int tiny_head, tiny_len;
+};
+__device__ HeadSplit split_heads(long long* off, int nheads, int grid, int cta, int lane) {
+  int ntiny = 0;
+  long long tbig = 0, tall = 0;
+  for (int base = 0; base < nheads; base += 32) {
+    const int i = base + lane;
+    const long long len = (i < nheads) ? off[i + 1] : 0;
+    const bool tiny = i < nheads && len <= kTinyLen;
+    ntiny += __popc(__ballot_sync(0xffffffffu, tiny));
+    long long big = tiny ? 0 : len, all = len;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      big += __shfl_xor_sync(0xffffffffu, big, o);
+      all += __shfl_xor_sync(0xffffffffu, all, o);
+    }
+    tbig += big;
+    tall += all;
+  }
+  const bool use = ntiny >= 1 && ntiny < nheads && 8 * ntiny <= grid && tbig >= grid - ntiny;
+  HeadSplit r;
+  r.ntiny = use ? ntiny : 0;
+  r.T = use ? tbig : tall;
+  r.P = min((long long)(grid - r.ntiny), r.T);
+  r.tiny_head = -1;
+  r.tiny_len = 0;
+  const long long k = (long long)cta - r.P;  // this CTA's rank among the tiny heads' CTAs
+  if (use && k >= 0 && k < ntiny) {
+    int seen = 0;
+    for (int base = 0; base < nheads; base += 32) {
+      const int i = base + lane;
+      const long long len = (i < nheads) ? off[i + 1] : 0;
+      const unsigned m = __ballot_sync(0xffffffffu, i < nheads && len <= kTinyLen);
+      const int here = __popc(m);
+      if (r.tiny_head < 0 && k < seen + here) {
+        const int l = __fns(m, 0, (int)(k - seen) + 1);  // lane of the (k - seen)-th set bit
+        r.tiny_head = base + l;
+        r.tiny_len = (int)__shfl_sync(0xffffffffu, len, l);
+      }
+      seen += here;
+    }
+  }
+  long long carry = 0;
+  for (int base = 0; base < nheads; base += 32) {  // inclusive scan, 32 heads at a time
+    const int i = base + lane;
+    const long long len = (i < nheads) ? off[i + 1] : 0;
+    long long x = (use && len <= kTinyLen) ? 0 : len;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const long long y = __shfl_up_sync(0xffffffffu, x, o);
+      if (lane >= o) x += y;
+    }
+    __syncwarp();  // every lane has read its size before any is overwritten
+    if (i < nheads) off[i + 1] = carry + x;
+    carry += __shfl_sync(0xffffffffu, x, 31);
+  }
+  if (lane == 0) off[0] = 0;
+  __syncwarp();
+  return r;
+}
+
 // The segments of this CTA's range, head by head, in order.
 struct Walk {
   const long long* off;
@@ -190,31 +265,33 @@ __global__ void __launch_bounds__(kAttendThreads, kAttendCtasPerSm) attend_kerne
     sOff[hd + 1] = len;
   }
   __syncthreads();
-  if (warp == 0) {  // inclusive scan of the lengths, 32 heads at a time
-    long long carry = 0;
-    for (int base = 0; base < nheads; base += 32) {
-      const int i = base + lane;
-      long long x = (i < nheads) ? sOff[i + 1] : 0;
-#pragma unroll
-      for (int o = 1; o < 32; o <<= 1) {
-        const long long y = __shfl_up_sync(0xffffffffu, x, o);
-        if (lane >= o) x += y;
-      }
-      if (i < nheads) sOff[i + 1] = carry + x;
-      carry += __shfl_sync(0xffffffffu, x, 31);
+  __shared__ long long sSplit[2];  // P, and the end of this CTA's laid-out coordinates
+  __shared__ int sRole;            // 0: a range of the laid-out sets, 1: a tiny head, 2: none
+  if (warp == 0) {
+    // P CTAs cut the laid-out sets, so every range is non-empty and the pieces of a head are
+    // exactly the CTAs c_first..c_last. A tiny head's CTA sees the sets as if its head were the
+    // only one: sizes 0 before it, its size from it on.
+    const HeadSplit sp = split_heads(sOff, nheads, (int)gridDim.x, (int)blockIdx.x, lane);
+    if (sp.tiny_head >= 0)
+      for (int h = lane; h <= nheads; h += 32) sOff[h] = (h > sp.tiny_head) ? sp.tiny_len : 0;
+    if (lane == 0) {
+      sSplit[0] = sp.P;
+      sSplit[1] = sp.tiny_head >= 0 ? sp.tiny_len : sp.T;
+      sRole = ((long long)blockIdx.x < sp.P) ? 0 : (sp.tiny_head >= 0 ? 1 : 2);
     }
-    if (lane == 0) sOff[0] = 0;
   }
   __syncthreads();
   pdl_launch_dependents();
-
-  // P = min(grid, T) CTAs take part, so every range is non-empty and the pieces of a head are
-  // exactly the CTAs c_first..c_last
-  const long long T = sOff[nheads];
-  const long long P = min((long long)gridDim.x, T);  // T >= 1: the launch covers >= 1 head
-  if ((long long)blockIdx.x >= P) return;
-  const long long t0 = floor_div((long long)blockIdx.x * T, P);
-  const long long t1 = floor_div(((long long)blockIdx.x + 1) * T, P);
+  if (sRole == 2) return;
+  long long t0, t1;
+  if (sRole == 0) {
+    const long long P = sSplit[0], T = sSplit[1];
+    t0 = floor_div((long long)blockIdx.x * T, P);
+    t1 = floor_div(((long long)blockIdx.x + 1) * T, P);
+  } else {
+    t0 = 0;
+    t1 = sSplit[1];
+  }
 
   // total tiles of this CTA (segments are few)
   int ktot = 0;
@@ -438,21 +515,16 @@ __global__ void __launch_bounds__(kMergeThreads) merge_kernel(const LayerArgs a,
   // only released by the attention launch after that point. Larger layers read the ranges the
   // attention launch recorded, after the wait.
   __shared__ long long mOff[kMergeDirectHeads + 1];
+  __shared__ long long mSplit[2];  // T and P of the attention launch's split
   const bool direct = nheads <= kMergeDirectHeads;
-  if (direct && warp == 0) {
-    long long carry = 0;
-    for (int base = 0; base < nheads; base += 32) {
-      const int i = base + lane;
-      long long x = (i < nheads) ? head_len(a, w, i, nullptr) : 0;
-#pragma unroll
-      for (int o = 1; o < 32; o <<= 1) {
-        const long long y = __shfl_up_sync(0xffffffffu, x, o);
-        if (lane >= o) x += y;
-      }
-      if (i < nheads) mOff[i + 1] = carry + x;
-      carry += __shfl_sync(0xffffffffu, x, 31);
+  if (direct && warp == 0) {  // the attention launch's split of the same sizes
+    for (int i = lane; i < nheads; i += 32) mOff[i + 1] = head_len(a, w, i, nullptr);
+    __syncwarp();
+    const HeadSplit sp = split_heads(mOff, nheads, a.attend_grid, -1, lane);
+    if (lane == 0) {
+      mSplit[0] = sp.T;
+      mSplit[1] = sp.P;
     }
-    if (lane == 0) mOff[0] = 0;
   }
   __syncthreads();
   pdl_wait();
@@ -461,8 +533,8 @@ __global__ void __launch_bounds__(kMergeThreads) merge_kernel(const LayerArgs a,
     const int hd = u / (a.G * 4), jq = (u >> 2) % a.G, qtr = u & 3;
     int c_first, n;
     if (direct) {
-      const long long T = mOff[nheads];
-      const long long P = min((long long)a.attend_grid, T);
+      if (mOff[hd + 1] == mOff[hd]) continue;  // a tiny head: its own CTA wrote it out
+      const long long T = mSplit[0], P = mSplit[1];
       c_first = (int)cta_of(mOff[hd], T, P);
       n = (int)cta_of(mOff[hd + 1] - 1, T, P) - c_first + 1;
     } else {
