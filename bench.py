@@ -33,10 +33,10 @@ sys.path.insert(0, ROOT)
 METRIC = "decode steps/s and effective HBM GB/s (% of roofline) at 128K–1M ctx"
 ROW_BYTES = 2 * 128 * 2      # one token's K and V rows (bf16, head_dim 128)
 # DRAM traffic of attend_kernel from one ncu capture (the attend_kernel summary under
-# profiles/): ctx_1m layer 2, 448.92 MB read + 3.65 MB written for 869 997 tokens x 512 B of
+# profiles/): ctx_1m layer 2, 448.90 MB read + 3.53 MB written for 869 997 tokens x 512 B of
 # algorithmic bytes. It is scaled to a bench launch by that launch's algorithmic bytes, and
 # reported only while the kernel's sources are the ones that were captured.
-ATTEND_NCU = {"source_sha256_16": "3ba9539208803253", "traffic_bytes": 448.9216e6 + 3.64672e6,
+ATTEND_NCU = {"source_sha256_16": "d0fb486cbd2e21fb", "traffic_bytes": 448.899328e6 + 3.533312e6,
               "algorithmic_bytes": 869997 * 512}
 IDX_BYTES = 16 * 2           # one token's indexer key (fp16, 16 dims)
 L2_FLUSH_BELOW = 1 << 30    # steps reading less than this are timed with L2 flushed
