@@ -41,7 +41,25 @@ struct CSmem {
   static constexpr size_t fin_off = ml_off + (size_t)kW * kMaxGroup * 2 * 4;  // m[8], l[8]
   static constexpr size_t total = fin_off + (size_t)kMaxGroup * 2 * 4;
 };
-static_assert((size_t)kW * kElems * 4 <= CSmem::o_off, "the warps' O fit in the stages");
+
+// A warp's O in its slot of the stages, rows of kSlotPitch floats: the pitch makes the MMA
+// fragment's stores (query heads 2t, 2t + 1 of lanes t = 0..3) fall in different banks.
+constexpr int kSlotPitch = kHeadDim + 4;
+constexpr int kSlotFloats = kMaxGroup * kSlotPitch;
+static_assert((size_t)kW * kSlotFloats * 4 <= CSmem::o_off, "the warps' O fit in the stages");
+
+// The shared::cluster address of `p` (this CTA's shared memory) in CTA `rank` of the cluster,
+// and a load from it.
+__device__ __forceinline__ uint32_t cluster_addr(const void* p, unsigned rank) {
+  uint32_t r;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(smem_u32(p)), "r"(rank));
+  return r;
+}
+__device__ __forceinline__ float ld_cluster_f32(uint32_t addr) {
+  float v;
+  asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(v) : "r"(addr));
+  return v;
+}
 
 }  // namespace
 
@@ -130,13 +148,13 @@ __global__ void __launch_bounds__(kT, 1) head_cluster_kernel(const LayerArgs a, 
     }
     const float f0 = (st.m0 == -INFINITY) ? 0.f : exp2f(st.m0 - M0);  // 0: a warp without tokens
     const float f1 = (st.m1 == -INFINITY) ? 0.f : exp2f(st.m1 - M1);
-    float* wo = reinterpret_cast<float*>(smem + CSmem::stage_off) + (size_t)warp * kElems;
+    float* wo = reinterpret_cast<float*>(smem + CSmem::stage_off) + (size_t)warp * kSlotFloats;
 #pragma unroll
     for (int mt = 0; mt < 8; ++mt) {
-      wo[(2 * t) * kHeadDim + 16 * mt + g] = st.acc[mt][0] * f0;
-      wo[(2 * t + 1) * kHeadDim + 16 * mt + g] = st.acc[mt][1] * f1;
-      wo[(2 * t) * kHeadDim + 16 * mt + g + 8] = st.acc[mt][2] * f0;
-      wo[(2 * t + 1) * kHeadDim + 16 * mt + g + 8] = st.acc[mt][3] * f1;
+      wo[(2 * t) * kSlotPitch + 16 * mt + g] = st.acc[mt][0] * f0;
+      wo[(2 * t + 1) * kSlotPitch + 16 * mt + g] = st.acc[mt][1] * f1;
+      wo[(2 * t) * kSlotPitch + 16 * mt + g + 8] = st.acc[mt][2] * f0;
+      wo[(2 * t + 1) * kSlotPitch + 16 * mt + g + 8] = st.acc[mt][3] * f1;
     }
   }
   if (tid < kMaxGroup) {  // the piece's (m, l) per query head, over the warps
@@ -156,9 +174,10 @@ __global__ void __launch_bounds__(kT, 1) head_cluster_kernel(const LayerArgs a, 
   {  // O of the piece: the warps' slots added in warp order
     const float* wo = reinterpret_cast<const float*>(smem + CSmem::stage_off);
     for (int e = tid; e < kElems; e += kT) {
+      const int at = (e / kHeadDim) * kSlotPitch + e % kHeadDim;
       float s = 0.f;
 #pragma unroll
-      for (int wq = 0; wq < kW; ++wq) s += wo[(size_t)wq * kElems + e];
+      for (int wq = 0; wq < kW; ++wq) s += wo[(size_t)wq * kSlotFloats + at];
       sO[e] = s;
     }
   }
@@ -166,23 +185,26 @@ __global__ void __launch_bounds__(kT, 1) head_cluster_kernel(const LayerArgs a, 
   // ---- the head: merge the cluster's pieces through distributed shared memory ---------------
   cluster.sync();  // every piece of the head is in its CTA's shared memory
   {
-    // every CTA's (m, l) per query head, one remote load per thread, all in flight together
+    // rank r writes output values [r E / C, (r + 1) E / C) of the G * 128 (E) of the head, at
+    // most 8 * 128 / kMinCluster = kT of them: one per thread. Every remote load of the merge
+    // is issued before any is used (one round trip): the thread's C values of its output, and
+    // one (m, l) value of one CTA per thread.
+    static_assert(kMaxGroup * kHeadDim / kMinCluster <= kT, "one output per thread");
     __shared__ float sAll[kMaxCluster][2 * kMaxGroup];
-    if (tid < C * 2 * kMaxGroup)
-      sAll[tid / (2 * kMaxGroup)][tid % (2 * kMaxGroup)] =
-          cluster.map_shared_rank(sFin, tid / (2 * kMaxGroup))[tid % (2 * kMaxGroup)];
-    __syncthreads();
-    // rank r writes output values [r E / C, (r + 1) E / C) of the G * 128 (E) of the head;
-    // with M = max_c m_c and f_c = 2^(m_c - M): out = sum_c f_c O_c / sum_c f_c l_c
     const int E = a.G * kHeadDim;
     const int e0 = (int)((long long)rank * E / C), e1 = (int)((long long)(rank + 1) * E / C);
-    float* out_head = a.out + ((size_t)b * a.Hq + (size_t)kvh * a.G) * kHeadDim;
-    for (int e = e0 + tid; e < e1; e += kT) {
-      const int jq = e / kHeadDim;
-      float oc[kMaxCluster];
+    const int e = e0 + tid;
+    float oc[kMaxCluster];
 #pragma unroll
-      for (int c = 0; c < kMaxCluster; ++c)  // the C remote values of this output, in flight together
-        oc[c] = (c < C) ? cluster.map_shared_rank(sO, c)[e] : 0.f;
+    for (int c = 0; c < kMaxCluster; ++c)
+      oc[c] = (e < e1 && c < C) ? ld_cluster_f32(cluster_addr(sO + e, (unsigned)c)) : 0.f;
+    if (tid < C * 2 * kMaxGroup) {
+      const int c = tid / (2 * kMaxGroup), i = tid % (2 * kMaxGroup);
+      sAll[c][i] = ld_cluster_f32(cluster_addr(sFin + i, (unsigned)c));
+    }
+    __syncthreads();
+    if (e < e1) {  // with M = max_c m_c and f_c = 2^(m_c - M): out = sum_c f_c O_c / sum_c f_c l_c
+      const int jq = e / kHeadDim;
       float M = -INFINITY;
 #pragma unroll
       for (int c = 0; c < kMaxCluster; ++c)
@@ -196,7 +218,7 @@ __global__ void __launch_bounds__(kT, 1) head_cluster_kernel(const LayerArgs a, 
         L += sAll[c][kMaxGroup + jq] * f;
         O += oc[c] * f;
       }
-      out_head[e] = O / L;
+      a.out[((size_t)b * a.Hq + (size_t)kvh * a.G) * kHeadDim + e] = O / L;
     }
     if (tid == 0 && rank == 0 && a.sel_count) a.sel_count[hd] = len;
   }
