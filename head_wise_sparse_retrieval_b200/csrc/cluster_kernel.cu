@@ -10,9 +10,10 @@
 // head): CTA rank r attends over ranks [r T / C, (r + 1) T / C) of the head's set with the decode
 // attention's tile step (attend_tile.cuh: 16-token tiles gathered by per-warp cp.async
 // pipelines, warp MMA with the G query heads as N = 8, online softmax). The CTA's warps merge
-// their (m, l, O) through shared memory, and the C pieces of the head are merged through
-// distributed shared memory, in a fixed order, by the cluster itself: rank r writes the r-th
-// C-th of the head's G * 128 output values. No partials go to global memory and no merge launch
+// their (m, l, O) through shared memory; the C pieces of the head are merged by the cluster
+// itself, in a fixed order: every CTA stores its piece to its slot in global memory, one cluster
+// barrier orders the stores before the reads, and rank r reads its share of every piece from L2
+// (one round trip) and writes the r-th C-th of the head's G * 128 output values. No merge launch
 // follows.
 #include <cooperative_groups.h>
 
@@ -47,19 +48,6 @@ struct CSmem {
 constexpr int kSlotPitch = kHeadDim + 4;
 constexpr int kSlotFloats = kMaxGroup * kSlotPitch;
 static_assert((size_t)kW * kSlotFloats * 4 <= CSmem::o_off, "the warps' O fit in the stages");
-
-// The shared::cluster address of `p` (this CTA's shared memory) in CTA `rank` of the cluster,
-// and a load from it.
-__device__ __forceinline__ uint32_t cluster_addr(const void* p, unsigned rank) {
-  uint32_t r;
-  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(smem_u32(p)), "r"(rank));
-  return r;
-}
-__device__ __forceinline__ float ld_cluster_f32(uint32_t addr) {
-  float v;
-  asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(v) : "r"(addr));
-  return v;
-}
 
 }  // namespace
 
@@ -182,48 +170,51 @@ __global__ void __launch_bounds__(kT, 1) head_cluster_kernel(const LayerArgs a, 
     }
   }
 
-  // ---- the head: merge the cluster's pieces through distributed shared memory ---------------
-  cluster.sync();  // every piece of the head is in its CTA's shared memory
+  // ---- the head: merge the cluster's pieces through global memory -------------------------
+  // Each CTA stores its piece (m, l, O) in its slot of cluster_parts; after one cluster barrier
+  // (release / acquire at cluster scope) rank r reads its share of every piece from L2 in one
+  // round trip. In early mode the previous launch may still read the slots: wait for it first.
+  if (a.early) pdl_wait();
+  float* part = w.cluster_parts + ((size_t)hd * C + rank) * kClusterPartFloats;
+  for (int i = tid; i < kElems / 4; i += kT)
+    reinterpret_cast<float4*>(part + 2 * kMaxGroup)[i] = reinterpret_cast<const float4*>(sO)[i];
+  if (tid < 2 * kMaxGroup) part[tid] = sFin[tid];
+  cluster.sync();  // every piece of the head is in global memory
   {
     // rank r writes output values [r E / C, (r + 1) E / C) of the G * 128 (E) of the head, at
-    // most 8 * 128 / kMinCluster = kT of them: one per thread. Every remote load of the merge
-    // is issued before any is used (one round trip): the thread's C values of its output, and
-    // one (m, l) value of one CTA per thread.
+    // most 8 * 128 / kMinCluster = kT of them: one per thread, with M = max_c m_c and
+    // f_c = 2^(m_c - M): out = sum_c f_c O_c / sum_c f_c l_c, the pieces in rank order
     static_assert(kMaxGroup * kHeadDim / kMinCluster <= kT, "one output per thread");
-    __shared__ float sAll[kMaxCluster][2 * kMaxGroup];
     const int E = a.G * kHeadDim;
     const int e0 = (int)((long long)rank * E / C), e1 = (int)((long long)(rank + 1) * E / C);
     const int e = e0 + tid;
-    float oc[kMaxCluster];
-#pragma unroll
-    for (int c = 0; c < kMaxCluster; ++c)
-      oc[c] = (e < e1 && c < C) ? ld_cluster_f32(cluster_addr(sO + e, (unsigned)c)) : 0.f;
-    if (tid < C * 2 * kMaxGroup) {
-      const int c = tid / (2 * kMaxGroup), i = tid % (2 * kMaxGroup);
-      sAll[c][i] = ld_cluster_f32(cluster_addr(sFin + i, (unsigned)c));
-    }
-    __syncthreads();
-    if (e < e1) {  // with M = max_c m_c and f_c = 2^(m_c - M): out = sum_c f_c O_c / sum_c f_c l_c
+    if (e < e1) {
       const int jq = e / kHeadDim;
+      const float* head_parts = w.cluster_parts + (size_t)hd * C * kClusterPartFloats;
+      float oc[kMaxCluster], mc[kMaxCluster], lc[kMaxCluster];
+#pragma unroll
+      for (int c = 0; c < kMaxCluster; ++c) {  // every load in flight together
+        const float* pc = head_parts + (size_t)c * kClusterPartFloats;
+        const bool in = c < C;
+        oc[c] = in ? __ldcg(pc + 2 * kMaxGroup + e) : 0.f;
+        mc[c] = in ? __ldcg(pc + jq) : -INFINITY;
+        lc[c] = in ? __ldcg(pc + kMaxGroup + jq) : 0.f;
+      }
       float M = -INFINITY;
 #pragma unroll
-      for (int c = 0; c < kMaxCluster; ++c)
-        if (c < C) M = fmaxf(M, sAll[c][jq]);
+      for (int c = 0; c < kMaxCluster; ++c) M = fmaxf(M, mc[c]);
       float L = 0.f, O = 0.f;
 #pragma unroll
       for (int c = 0; c < kMaxCluster; ++c) {
-        const float mc = (c < C) ? sAll[c][jq] : -INFINITY;
-        if (mc == -INFINITY) continue;  // a CTA without tokens (heads shorter than the cluster)
-        const float f = exp2f(mc - M);
-        L += sAll[c][kMaxGroup + jq] * f;
+        if (mc[c] == -INFINITY) continue;  // a CTA without tokens, or past the cluster
+        const float f = exp2f(mc[c] - M);
+        L += lc[c] * f;
         O += oc[c] * f;
       }
       a.out[((size_t)b * a.Hq + (size_t)kvh * a.G) * kHeadDim + e] = O / L;
     }
     if (tid == 0 && rank == 0 && a.sel_count) a.sel_count[hd] = len;
   }
-  cluster.sync();  // no CTA leaves while another still reads its shared memory
-  if (a.early) pdl_wait();
 }
 
 }  // namespace rtp

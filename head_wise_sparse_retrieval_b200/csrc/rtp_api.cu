@@ -122,12 +122,13 @@ rtp_status check_config(const rtp_config* c) {
 }
 
 struct WsPlan {
-  size_t off[20];
+  size_t off[21];
   size_t total;
 };
 
 // Byte offsets of the workspace arrays (each 256-byte aligned).
-WsPlan plan_workspace(const rtp_config* c, int attend_grid, int select_grid, int fused_grid) {
+WsPlan plan_workspace(const rtp_config* c, int attend_grid, int select_grid, int fused_grid,
+                      int cluster_ctas) {
   const size_t slots = (size_t)c->batch * c->num_kv_heads;
   const size_t nmax = round_up((size_t)c->max_ctx, 64);  // per-slot stride (16-byte loads)
   const bool fused = slots <= (size_t)kFusedMaxHeads;
@@ -152,6 +153,7 @@ WsPlan plan_workspace(const rtp_config* c, int attend_grid, int select_grid, int
       fused ? slots * 4 : 0,                 // 17 smax_key
       fused ? slots * (nmax / 64) * 8 : 0,   // 18 sel_bits
       fused ? (slots * fused_grid + fused_grid + slots) * kPartFloats * 4 : 0,  // 19 pieces
+      (size_t)cluster_ctas * kClusterPartFloats * 4,  // 20 cluster_parts (B*Hkv*C <= #SMs)
   };
   WsPlan p{};
   size_t at = 0;
@@ -396,7 +398,7 @@ size_t rtp_workspace_bytes(const rtp_config* cfg) {
   int dev = 0, sms = 148;
   if (cudaGetDevice(&dev) == cudaSuccess)
     cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-  return plan_workspace(cfg, sms * kAttendCtasPerSm, sms * kMaxSelectCtasPerSm, sms).total;
+  return plan_workspace(cfg, sms * kAttendCtasPerSm, sms * kMaxSelectCtasPerSm, sms, sms).total;
 }
 
 rtp_status rtp_create(const rtp_config* cfg, int device, rtp_handle** out) {
@@ -438,7 +440,7 @@ rtp_status rtp_create(const rtp_config* cfg, int device, rtp_handle** out) {
   if (sel_per_sm > kMaxSelectCtasPerSm) sel_per_sm = kMaxSelectCtasPerSm;
   h->select_grid = h->num_sms * sel_per_sm;  // cooperative: every CTA resident at once
   h->fused_grid = h->num_sms;  // one CTA per SM
-  const WsPlan p = plan_workspace(cfg, h->attend_grid, h->select_grid, h->fused_grid);
+  const WsPlan p = plan_workspace(cfg, h->attend_grid, h->select_grid, h->fused_grid, h->num_sms);
   const size_t L = (size_t)cfg->num_layers, B = (size_t)cfg->batch;
   const size_t q_bytes = L * B * cfg->num_q_heads * kHeadDim * 2;
   const size_t qi_bytes = L * B * cfg->num_kv_heads * kIdxDim * 2;
@@ -477,6 +479,7 @@ rtp_status rtp_create(const rtp_config* cfg, int device, rtp_handle** out) {
   w.sel_n = reinterpret_cast<int*>(base + p.off[10]);
   w.grid_bar = reinterpret_cast<unsigned*>(base + p.off[11]);
   w.head_pieces = reinterpret_cast<int2*>(base + p.off[13]);
+  w.cluster_parts = reinterpret_cast<float*>(base + p.off[20]);
   w.partials = reinterpret_cast<float*>(base + p.off[14]);
   w.status = reinterpret_cast<unsigned*>(base + p.off[15]);
   h->hist_cnt = reinterpret_cast<unsigned*>(base + p.off[16]);

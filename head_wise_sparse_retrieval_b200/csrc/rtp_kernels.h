@@ -33,6 +33,7 @@ struct Workspace {
   unsigned* grid_bar;             // [0]: grid barrier counter of the selection kernel
   float* partials;                // [(attend_ctas + B*Hkv)][kPartFloats]  piece of CTA c, head h at c + h
   int2* head_pieces;              // [B*Hkv]                 first and last attention CTA of a head
+  float* cluster_parts;           // [B*Hkv*C][kClusterPartFloats] pieces of the cluster launch
   unsigned* status;               // [1] RTP_DEV_* bits
   int ld;                         // per-slot stride of scores / sel_idx: max_ctx rounded up to 64
 };
@@ -94,6 +95,7 @@ constexpr int kClusterDepth = 3;                         // cp.async stages per 
 constexpr int kMaxCluster = 16;                          // CTAs of one cluster (non-portable > 8)
 constexpr int kMinCluster = 4;                           // below this the split launches serve better
 constexpr int kClusterMaxSet = 65536;                    // window + sinks of a cluster layer
+constexpr int kClusterPartFloats = 2 * 8 + 8 * 128;      // a cluster CTA's piece: m[8], l[8], O
 __global__ void head_cluster_kernel(const LayerArgs a, const Workspace w);
 size_t cluster_smem_bytes();
 
