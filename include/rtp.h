@@ -147,7 +147,7 @@ typedef struct {
  * kernels: the selection, the attention of every head (split over the SMs), and the merge of
  * the split heads. A layer of local heads only is one kernel when the handle's B * Hkv leaves at
  * least 4 SMs per KV head (and window + sinks <= 65536): one thread-block cluster per KV head,
- * whose CTAs merge the head's pieces in distributed shared memory; otherwise attention and
+ * whose CTAs merge the head's pieces inside the launch; otherwise attention and
  * merge as above. Asynchronous: no host synchronisation,
  * no allocation, capturable in a CUDA graph (the mask is read on the host at call time and the
  * launch shapes depend only on cfg and the mask). Errors (nothing enqueued): RTP_ERR_INVALID_ARG

@@ -131,8 +131,8 @@ def test_small_window_and_no_sinks():
 ])
 def test_local_only_layers(B, Hkv, G, seq_lens):
     """Layers without retrieval heads run as one launch of one or more thread-block clusters
-    per KV head when the SMs allow (their pieces merged in distributed shared memory, and across
-    clusters by a last-arriver ticket), else as the split attention and merge launches; every
+    per KV head when the SMs allow (the cluster merges its CTAs' pieces itself, through L2 after
+    a cluster barrier), else as the split attention and merge launches; every
     head against the oracle, with the cache past each context poisoned, bit-identical reruns,
     and the launch count of the path that ran."""
     p = W.custom(batch=B, num_q_heads=Hkv * G, num_kv_heads=Hkv, seq_lens=seq_lens,

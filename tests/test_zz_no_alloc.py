@@ -9,7 +9,7 @@ look-up of the array's address, and check:
   * each result against the handle-based entry point's: bit-identical to rtp_dense_decode (the
     same attention and merge kernels on the same grid), and for local heads within the parity
     bars of rtp_decode_step, which runs a layer of local heads as one cluster launch that merges
-    in distributed shared memory instead (another summation order), as well as against the
+    inside the launch instead (another summation order), as well as against the
     oracle;
   * the caching allocator's allocated and reserved bytes do not move across the two calls;
   * a handle created earlier for a larger layer still decodes correctly afterwards (the
