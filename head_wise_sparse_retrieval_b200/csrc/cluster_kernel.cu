@@ -32,22 +32,19 @@ constexpr int kD = kClusterDepth;
 constexpr int kT = kW * 32;
 constexpr int kElems = kMaxGroup * kHeadDim;  // one head's output values (8 query heads x 128)
 
-// Shared memory: the warps' stages, then the CTA's piece: O (unnormalised, [8][128]) and, per
-// query head, the piece's maximum m (log2 domain) and sum l. At the end the stages hold the
-// warps' rescaled O for the CTA-level merge.
+// Shared memory: the warps' stages, then each warp's maximum m (log2 domain) and sum l per query
+// head. At the end the stages hold the warps' rescaled O for the CTA-level merge.
 struct CSmem {
   static constexpr size_t stage_off = 0;
-  static constexpr size_t o_off = (size_t)kW * kD * kWarpStage;
-  static constexpr size_t ml_off = o_off + (size_t)kElems * 4;   // per warp: m[8], l[8]
-  static constexpr size_t fin_off = ml_off + (size_t)kW * kMaxGroup * 2 * 4;  // m[8], l[8]
-  static constexpr size_t total = fin_off + (size_t)kMaxGroup * 2 * 4;
+  static constexpr size_t ml_off = (size_t)kW * kD * kWarpStage;  // per warp: m[8], l[8]
+  static constexpr size_t total = ml_off + (size_t)kW * kMaxGroup * 2 * 4;
 };
 
 // A warp's O in its slot of the stages, rows of kSlotPitch floats: the pitch makes the MMA
 // fragment's stores (query heads 2t, 2t + 1 of lanes t = 0..3) fall in different banks.
 constexpr int kSlotPitch = kHeadDim + 4;
 constexpr int kSlotFloats = kMaxGroup * kSlotPitch;
-static_assert((size_t)kW * kSlotFloats * 4 <= CSmem::o_off, "the warps' O fit in the stages");
+static_assert((size_t)kW * kSlotFloats * 4 <= CSmem::ml_off, "the warps' O fit in the stages");
 
 }  // namespace
 
@@ -55,9 +52,7 @@ size_t cluster_smem_bytes() { return CSmem::total; }
 
 __global__ void __launch_bounds__(kT, 1) head_cluster_kernel(const LayerArgs a, const Workspace w) {
   extern __shared__ __align__(128) unsigned char smem[];
-  float* sO = reinterpret_cast<float*>(smem + CSmem::o_off);
   float* sML = reinterpret_cast<float*>(smem + CSmem::ml_off);
-  float* sFin = reinterpret_cast<float*>(smem + CSmem::fin_off);
   cg::cluster_group cluster = cg::this_cluster();
   const int C = (int)cluster.num_blocks();
   const int rank = (int)cluster.block_rank();
@@ -65,8 +60,8 @@ __global__ void __launch_bounds__(kT, 1) head_cluster_kernel(const LayerArgs a, 
   const int b = hd / a.Hkv, kvh = hd - b * a.Hkv;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
 
-  // Nothing here is read by the launch before (the previous layer's merge); when the caller
-  // vouches that the inputs are ready, the wait moves to the end, so that this launch still
+  // When the caller vouches that the inputs are ready, the wait moves to just before the first
+  // store to the pieces' slots, which the launch before may still read; this launch then still
   // completes after its predecessor.
   if (!a.early) pdl_wait();
   int N = __ldg(a.seq_lens + b);
@@ -145,6 +140,14 @@ __global__ void __launch_bounds__(kT, 1) head_cluster_kernel(const LayerArgs a, 
       wo[(2 * t + 1) * kSlotPitch + 16 * mt + g + 8] = st.acc[mt][3] * f1;
     }
   }
+  __syncthreads();  // every warp's slot is written
+
+  // ---- the head: merge the cluster's pieces through global memory -------------------------
+  // Each CTA stores its piece (m, l, O) in its slot of cluster_parts; after one cluster barrier
+  // (release / acquire at cluster scope) rank r reads its share of every piece from L2 in one
+  // round trip. In early mode the launch before may still read the slots: wait for it first.
+  if (a.early) pdl_wait();
+  float* part = w.cluster_parts + ((size_t)hd * C + rank) * kClusterPartFloats;
   if (tid < kMaxGroup) {  // the piece's (m, l) per query head, over the warps
     float M = -INFINITY;
 #pragma unroll
@@ -155,30 +158,19 @@ __global__ void __launch_bounds__(kT, 1) head_cluster_kernel(const LayerArgs a, 
       const float mw = sML[(wq * kMaxGroup + tid) * 2];
       if (mw != -INFINITY) L += sML[(wq * kMaxGroup + tid) * 2 + 1] * exp2f(mw - M);
     }
-    sFin[tid] = M;
-    sFin[kMaxGroup + tid] = L;
+    part[tid] = M;
+    part[kMaxGroup + tid] = L;
   }
-  __syncthreads();
-  {  // O of the piece: the warps' slots added in warp order
+  {  // O of the piece: the warps' slots added in warp order, stored to the slot directly
     const float* wo = reinterpret_cast<const float*>(smem + CSmem::stage_off);
     for (int e = tid; e < kElems; e += kT) {
       const int at = (e / kHeadDim) * kSlotPitch + e % kHeadDim;
-      float s = 0.f;
+      float v = 0.f;
 #pragma unroll
-      for (int wq = 0; wq < kW; ++wq) s += wo[(size_t)wq * kSlotFloats + at];
-      sO[e] = s;
+      for (int wq = 0; wq < kW; ++wq) v += wo[(size_t)wq * kSlotFloats + at];
+      part[2 * kMaxGroup + e] = v;
     }
   }
-
-  // ---- the head: merge the cluster's pieces through global memory -------------------------
-  // Each CTA stores its piece (m, l, O) in its slot of cluster_parts; after one cluster barrier
-  // (release / acquire at cluster scope) rank r reads its share of every piece from L2 in one
-  // round trip. In early mode the previous launch may still read the slots: wait for it first.
-  if (a.early) pdl_wait();
-  float* part = w.cluster_parts + ((size_t)hd * C + rank) * kClusterPartFloats;
-  for (int i = tid; i < kElems / 4; i += kT)
-    reinterpret_cast<float4*>(part + 2 * kMaxGroup)[i] = reinterpret_cast<const float4*>(sO)[i];
-  if (tid < 2 * kMaxGroup) part[tid] = sFin[tid];
   cluster.sync();  // every piece of the head is in global memory
   {
     // rank r writes output values [r E / C, (r + 1) E / C) of the G * 128 (E) of the head, at
